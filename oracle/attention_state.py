@@ -1,0 +1,413 @@
+"""Plain float64 oracle of the attention-state reuse step (test infrastructure).
+
+TEST INFRASTRUCTURE ONLY -- see the package docstring.  Slow and obviously
+correct: numpy float64, a library matmul as the only "primitive", no blocking
+beyond the 128-row query/key tiles that the plan itself is defined on.
+
+Sources (cited by page title and the part of the page):
+  [DT]  "DiTango: Cost-Effective Parallel Diffusion Generation with Selective
+        Attention State Reuse" -- the attention-state definition (Eq. 1-3),
+        composability of states (Eq. 4), the selective compute/reuse mechanism
+        (Fig. 6 example, CP=4, rank 0), grouping and anchor steps (Eq. 8-9,
+        Algorithm 1).  The display equations were lost from the page text;
+        the readings below are the plainest ones the surrounding prose allows.
+  [DFA] "DiTFastAttn: Attention Compression for Diffusion Transformer Models"
+        (summary page, "Approach"): window attention plus a cached
+        full-minus-window residual.
+
+Readings taken where the pages are silent (each also listed in the design
+notes of the repository):
+  * state = (OUT, LSE) with OUT normalised by the partition's own softmax
+    denominator and LSE the natural-log log-sum-exp of the scaled logits;
+  * softmax scale 1/sqrt(D) on q.k;
+  * partitions are contiguous: c = ceil(S/P), partition k = [k c, min((k+1)c, S));
+  * query tiles are 128-row, partition-local; every row of a tile shares the
+    tile's plan row;
+  * proximity plan: for query partition q the r partitions farthest from q
+    are reused, ties broken towards the lower index; q itself is always
+    computed; step 1 is an anchor (everything computed);
+  * window: key j is in the window of query i iff |i - j| <= W // 2 on the
+    flattened token order, no wrap-around.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+TILE = 128
+REUSE = 0
+COMPUTE = 1
+
+MODE_ALL_COMPUTE = 0
+MODE_PROXIMITY = 1
+MODE_ALL_REUSE = 2
+MODE_EXPLICIT = 3
+MODE_WINDOW = 4
+
+__all__ = [
+    "TILE", "REUSE", "COMPUTE", "MODE_ALL_COMPUTE", "MODE_PROXIMITY",
+    "MODE_ALL_REUSE", "MODE_EXPLICIT", "MODE_WINDOW", "CacheEmpty",
+    "widen_bf16", "round_bf16", "partitions", "query_tiles", "n_kv_tiles",
+    "attention_state", "identity_state", "compose", "compose_n",
+    "proximity_row", "build_plan", "window_in", "StateCache",
+    "partition_step", "window_step", "softmax_scale",
+]
+
+
+class CacheEmpty(Exception):
+    """A REUSE entry points at a cache slot that has never been written."""
+
+
+# ----------------------------------------------------------------------------
+# bf16 helpers (exact widening; RNE narrowing of the final output)
+# ----------------------------------------------------------------------------
+
+def widen_bf16(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> float64, exactly."""
+    u = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return u.view(np.float32).astype(np.float64)
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """float64 -> nearest bf16 value (ties to even), returned as float64."""
+    f = np.ascontiguousarray(x, dtype=np.float64)
+    # exact two-step: to float32 may double-round, so round from float64 bits.
+    out = np.empty_like(f)
+    flat = f.reshape(-1)
+    o = out.reshape(-1)
+    for i in range(0, flat.size, 1 << 20):
+        blk = flat[i:i + (1 << 20)]
+        m, e = np.frexp(blk)            # blk = m * 2**e, 0.5 <= |m| < 1
+        q = np.ldexp(np.round(np.ldexp(m, 8)), e - 8)   # 8 significant bits
+        o[i:i + (1 << 20)] = q
+    return out
+
+
+def softmax_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)
+
+
+# ----------------------------------------------------------------------------
+# Geometry  [DT] context partitioning (contiguous sequence slabs)
+# ----------------------------------------------------------------------------
+
+def partitions(S: int, P: int) -> List[Tuple[int, int]]:
+    """Contiguous partitions [start, end) of the token sequence, P of them."""
+    c = -(-S // P) if S > 0 else 0
+    return [(min(k * c, S), min((k + 1) * c, S)) for k in range(P)]
+
+
+def query_tiles(S: int, P: int, window: int = 0) -> List[Tuple[int, int, int]]:
+    """Query tiles (partition index, first row, end row), 128 rows each,
+    partition-local.  Window mode has one partition spanning the sequence."""
+    parts = [(0, S)] if window > 0 else partitions(S, P)
+    out = []
+    for k, (a, b) in enumerate(parts):
+        for q0 in range(a, b, TILE):
+            out.append((k, q0, min(q0 + TILE, b)))
+    return out
+
+
+def n_kv_tiles(a: int, b: int) -> int:
+    return -(-(b - a) // TILE) if b > a else 0
+
+
+# ----------------------------------------------------------------------------
+# [DT] attention state (Eq. 1-3) and its composition (Eq. 4)
+# ----------------------------------------------------------------------------
+
+def identity_state(n: int, D: int) -> Tuple[np.ndarray, np.ndarray]:
+    """State of an empty key set: OUT = 0, LSE = -inf (the unit of compose)."""
+    return np.zeros((n, D)), np.full(n, -np.inf)
+
+
+def attention_state(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                    keep: Optional[np.ndarray] = None):
+    """Partial attention of queries q [n,D] over keys k,v [m,D].
+
+    s_ij = scale * q_i . k_j ;  m_i = max_j s_ij ;  l_i = sum_j exp(s_ij - m_i)
+    OUT_i = sum_j exp(s_ij - m_i) v_j / l_i ;  LSE_i = m_i + ln l_i
+    ``keep`` (bool [n,m]) removes pairs from the key set; a row whose key set
+    is empty gets the identity state.
+    """
+    n, D = q.shape[0], v.shape[1] if v.ndim == 2 else q.shape[1]
+    if k.shape[0] == 0:
+        return identity_state(n, D)
+    s = (q @ k.T) * scale
+    if keep is not None:
+        s = np.where(keep, s, -np.inf)
+    m = s.max(axis=1)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    e = np.exp(s - m_safe[:, None])
+    l = e.sum(axis=1)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = (e @ v) / l[:, None]
+        lse = m_safe + np.log(l)
+    out[empty] = 0.0
+    lse[empty] = -np.inf
+    return out, lse
+
+
+def compose(a, b):
+    """Binary composition of two states of the same rows.
+
+    L = M + ln(e^(L1-M) + e^(L2-M)),  M = max(L1, L2)
+    OUT = e^(L1-L) OUT1 + e^(L2-L) OUT2;  (0, -inf) when both are empty.
+    """
+    (o1, l1), (o2, l2) = a, b
+    M = np.maximum(l1, l2)
+    both_empty = ~np.isfinite(M)
+    Ms = np.where(both_empty, 0.0, M)
+    w1 = np.exp(l1 - Ms)
+    w2 = np.exp(l2 - Ms)
+    with np.errstate(divide="ignore"):
+        L = Ms + np.log(w1 + w2)
+    L = np.where(both_empty, -np.inf, L)
+    Ls = np.where(both_empty, 0.0, L)
+    c1 = np.where(both_empty, 0.0, np.exp(l1 - Ls))
+    c2 = np.where(both_empty, 0.0, np.exp(l2 - Ls))
+    return c1[:, None] * o1 + c2[:, None] * o2, L
+
+
+def compose_n(states: Sequence[Tuple[np.ndarray, np.ndarray]]):
+    """N-way composition: one max over all N LSEs, then one weighted pass."""
+    L = np.stack([s[1] for s in states])            # [N, n]
+    M = L.max(axis=0)
+    empty = ~np.isfinite(M)
+    Ms = np.where(empty, 0.0, M)
+    w = np.exp(L - Ms[None, :])                      # [N, n]
+    tot = w.sum(axis=0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        Lout = np.where(empty, -np.inf, Ms + np.log(tot))
+        c = np.where(empty[None, :], 0.0, w / tot[None, :])
+    out = np.zeros_like(states[0][0])
+    for i, s in enumerate(states):
+        out += c[i][:, None] * s[0]
+    return out, Lout
+
+
+# ----------------------------------------------------------------------------
+# Plans  [DT] selective compute/reuse (Fig. 6), spatial proximity (Fig. 5a),
+#        anchor steps; [DFA] window + residual as a two-key-set plan
+# ----------------------------------------------------------------------------
+
+def proximity_row(q: int, P: int, r: int) -> np.ndarray:
+    """Plan row of query partition q: the r farthest partitions are reused
+    (lower index first among equal distances); q itself is always computed."""
+    row = np.full(P, COMPUTE, dtype=np.uint8)
+    others = sorted((k for k in range(P) if k != q), key=lambda k: (-abs(q - k), k))
+    for k in others[:r]:
+        row[k] = REUSE
+    return row
+
+
+def window_in(i: np.ndarray, j: np.ndarray, W: int) -> np.ndarray:
+    """[DFA] key j lies in the window of query i iff |i - j| <= W // 2."""
+    return np.abs(i[:, None] - j[None, :]) <= (W // 2)
+
+
+def _window_tile_blocks(q0: int, q1: int, S: int, W: int):
+    """(band blocks, total blocks) of one query tile: a 128x128 block is in the
+    band iff at least one of its (query, key) pairs lies in the window."""
+    hw = W // 2
+    nkt = n_kv_tiles(0, S)
+    band = 0
+    for t in range(nkt):
+        a, b = t * TILE, min(t * TILE + TILE, S) - 1
+        if a - (q1 - 1) <= hw and q0 - b <= hw:
+            band += 1
+    return band, nkt
+
+
+def _window_pairs(q0: int, q1: int, S: int, W: int) -> int:
+    hw = W // 2
+    tot = 0
+    for i in range(q0, q1):
+        tot += min(S - 1, i + hw) - max(0, i - hw) + 1
+    return tot
+
+
+def build_plan(mode: int, H: int, S: int, D: int, P: int, step: int,
+               r: int = 0, window: int = 0,
+               stamps: Optional[np.ndarray] = None,
+               explicit: Optional[np.ndarray] = None):
+    """Plan, block counts, algorithmic FLOPs and updated stamps of one step.
+
+    Returns ``(plan uint8 [nqt][nseg], counts, stamps')`` where nseg = P (2 in
+    window mode: key sets "window" and "complement"), counts =
+    {computed_blocks, skipped_blocks, computed_flops}.  Step 1 of the proximity
+    and window modes is an anchor: everything is computed.  A REUSE entry whose
+    stamp is -1 raises ``CacheEmpty``; COMPUTE entries get stamp = step.
+    """
+    tiles = query_tiles(S, P, window)
+    nqt = len(tiles)
+    if mode == MODE_WINDOW:
+        nseg = 2
+        plan = np.full((nqt, 2), COMPUTE, dtype=np.uint8)
+        if step > 1:
+            plan[:, 1] = REUSE
+    else:
+        nseg = P
+        plan = np.empty((nqt, P), dtype=np.uint8)
+        for t, (kq, _, _) in enumerate(tiles):
+            if mode == MODE_ALL_COMPUTE or (mode == MODE_PROXIMITY and step <= 1):
+                plan[t] = COMPUTE
+            elif mode == MODE_PROXIMITY:
+                plan[t] = proximity_row(kq, P, r)
+            elif mode == MODE_ALL_REUSE:
+                plan[t] = REUSE
+            elif mode == MODE_EXPLICIT:
+                plan[t] = np.asarray(explicit, dtype=np.uint8).reshape(nqt, P)[t]
+            else:
+                raise ValueError(mode)
+    st = (np.full((nqt, nseg), -1, dtype=np.int32) if stamps is None
+          else np.array(stamps, dtype=np.int32).reshape(nqt, nseg).copy())
+    if np.any((plan == REUSE) & (st < 0)):
+        raise CacheEmpty("REUSE of a cache slot that was never written")
+    st[plan == COMPUTE] = step
+
+    parts = partitions(S, P)
+    cb = sb = fl = 0
+    for t, (_, q0, q1) in enumerate(tiles):
+        if mode == MODE_WINDOW:
+            band, nkt = _window_tile_blocks(q0, q1, S, window)
+            if plan[t, 1] == COMPUTE:
+                cb += H * nkt
+                fl += 4 * H * D * (q1 - q0) * S
+            else:
+                cb += H * band
+                sb += H * (nkt - band)
+                fl += 4 * H * D * _window_pairs(q0, q1, S, window)
+        else:
+            for k, (a, b) in enumerate(parts):
+                nb = H * n_kv_tiles(a, b)
+                if plan[t, k] == COMPUTE:
+                    cb += nb
+                    fl += 4 * H * D * (q1 - q0) * (b - a)
+                else:
+                    sb += nb
+    counts = {"computed_blocks": cb, "skipped_blocks": sb, "computed_flops": fl}
+    return plan, counts, st
+
+
+# ----------------------------------------------------------------------------
+# One denoising step of the method, for all rows or for a sample of rows
+# ----------------------------------------------------------------------------
+
+class StateCache:
+    """Per-(KV partition, head) cached states of query rows.
+
+    ``out[k][h]`` is a dict row -> (OUT [D], LSE) for the rows tracked.  Rows
+    are independent, so a sampled subset of rows can be followed through a
+    whole schedule exactly.
+    """
+
+    def __init__(self):
+        self.slots: Dict[Tuple[int, int, int], Tuple[np.ndarray, float]] = {}
+
+    def put(self, k, h, rows, out, lse):
+        for i, r in enumerate(rows):
+            self.slots[(k, h, int(r))] = (out[i].copy(), float(lse[i]))
+
+    def get(self, k, h, rows, D):
+        out = np.empty((len(rows), D))
+        lse = np.empty(len(rows))
+        for i, r in enumerate(rows):
+            o, l = self.slots[(k, h, int(r))]
+            out[i], lse[i] = o, l
+        return out, lse
+
+
+def _tile_of_rows(tiles, rows):
+    starts = np.array([t[1] for t in tiles])
+    return np.searchsorted(starts, rows, side="right") - 1
+
+
+def partition_step(Q: np.ndarray, K: np.ndarray, V: np.ndarray, plan: np.ndarray,
+                   S: int, P: int, cache: StateCache,
+                   heads: Optional[Sequence[int]] = None,
+                   rows: Optional[np.ndarray] = None):
+    """[DT] One step: (O, LSE)_q = compose over k of (fresh if COMPUTE else
+    cached); fresh states overwrite their slots afterwards.
+
+    Q, K, V: float64 [H][S][D] (or bf16 bits, widened here).  Returns
+    ``(O, LSE, fresh)`` for the selected heads x rows, O in float64 (the
+    caller rounds to bf16), ``fresh`` a dict (k, h) -> (rows, OUT, LSE) of the
+    states computed this step.  ``cache`` is updated in place.
+    """
+    if Q.dtype == np.uint16:
+        Q, K, V = widen_bf16(Q), widen_bf16(K), widen_bf16(V)
+    H, _, D = Q.shape
+    heads = list(range(H)) if heads is None else list(heads)
+    rows = np.arange(S) if rows is None else np.asarray(rows)
+    tiles = query_tiles(S, P)
+    parts = partitions(S, P)
+    tix = _tile_of_rows(tiles, rows)
+    scale = softmax_scale(D)
+    O = np.zeros((len(heads), len(rows), D))
+    L = np.zeros((len(heads), len(rows)))
+    fresh = {}
+    for hi, h in enumerate(heads):
+        pending = []
+        for t in np.unique(tix):
+            sel = np.nonzero(tix == t)[0]
+            rs = rows[sel]
+            states = []
+            for k, (a, b) in enumerate(parts):
+                if plan[t, k] == COMPUTE:
+                    st = attention_state(Q[h, rs], K[h, a:b], V[h, a:b], scale)
+                    pending.append((k, h, rs, st))
+                    fresh.setdefault((k, h), []).append((rs, st))
+                else:
+                    st = cache.get(k, h, rs, D)
+                states.append(st)
+            o, l = states[0]
+            for st in states[1:]:
+                o, l = compose((o, l), st)
+            O[hi, sel], L[hi, sel] = o, l
+        for k, h_, rs, st in pending:
+            cache.put(k, h_, rs, st[0], st[1])
+    return O, L, fresh
+
+
+def window_step(Q: np.ndarray, K: np.ndarray, V: np.ndarray, W: int,
+                make_residual: bool, R: Optional[Dict[Tuple[int, int], np.ndarray]],
+                heads: Optional[Sequence[int]] = None,
+                rows: Optional[np.ndarray] = None):
+    """[DFA] window attention with a cached residual.
+
+    make_residual (anchor step): full = window (+) complement,
+    R = OUT_full - OUT_window, O = OUT_full, LSE = LSE_full.
+    otherwise: O = OUT_window + R, LSE = LSE_window.
+    R is a dict (h, row) -> [D] float64, updated in place when made.
+    """
+    if Q.dtype == np.uint16:
+        Q, K, V = widen_bf16(Q), widen_bf16(K), widen_bf16(V)
+    H, S, D = Q.shape
+    heads = list(range(H)) if heads is None else list(heads)
+    rows = np.arange(S) if rows is None else np.asarray(rows)
+    scale = softmax_scale(D)
+    keys = np.arange(S)
+    O = np.zeros((len(heads), len(rows), D))
+    L = np.zeros((len(heads), len(rows)))
+    for hi, h in enumerate(heads):
+        for i0 in range(0, len(rows), TILE):
+            rs = rows[i0:i0 + TILE]
+            inside = window_in(rs, keys, W)
+            win = attention_state(Q[h, rs], K[h], V[h], scale, keep=inside)
+            if make_residual:
+                comp = attention_state(Q[h, rs], K[h], V[h], scale, keep=~inside)
+                full = compose(win, comp)
+                res = full[0] - win[0]
+                for j, r in enumerate(rs):
+                    R[(h, int(r))] = res[j].copy()
+                O[hi, i0:i0 + len(rs)], L[hi, i0:i0 + len(rs)] = full
+            else:
+                res = np.stack([R[(h, int(r))] for r in rs])
+                O[hi, i0:i0 + len(rs)] = win[0] + res
+                L[hi, i0:i0 + len(rs)] = win[1]
+    return O, L
