@@ -1,0 +1,181 @@
+/*
+ * dt.h -- C ABI of the partitioned attention-state library (libdt.so).
+ *
+ * One denoising step of a Diffusion Transformer's full attention, split over P
+ * contiguous context partitions.  For every (query tile, KV partition) pair a
+ * per-step plan either COMPUTEs a fresh partial attention state or REUSEs the
+ * state of that pair cached at an earlier step; the output is the
+ * log-sum-exp weighted composition of all P states, and fresh states
+ * overwrite their cache slots.  Window attention with a cached
+ * full-minus-window residual is a second plan mode on the same machinery.
+ *
+ * Sources: "DiTango: Cost-Effective Parallel Diffusion Generation with
+ * Selective Attention State Reuse" (attention state, Eq. 1-3; composition,
+ * Eq. 4; selective compute and reuse, Fig. 6; anchor steps) and
+ * "DiTFastAttn: Attention Compression for Diffusion Transformer Models"
+ * (summary page, Approach: window attention with residual sharing).
+ *
+ * Conventions for every entry point
+ *   - returns an int status: DT_OK (0) or a negative DT_ERR_* code; no C++
+ *     exception crosses this boundary;
+ *   - the caller owns and allocates every buffer; the library allocates no
+ *     device or host memory (tensor memory inside a kernel aside);
+ *   - device work is enqueued asynchronously on the caller's stream
+ *     (cudaStream_t passed as void*; NULL = legacy default stream);
+ *   - device pointers must be 16-byte aligned; kernels report device-side
+ *     errors by writing a DT_ERR_* code into *d_status (int32, device memory,
+ *     caller-zeroed), which the caller reads after synchronising;
+ *   - tensors are dense, row-major, batch 1:
+ *       Q, K, V, O           bf16  [H][S][D]
+ *       L (final LSE)        fp32  [H][S]
+ *       cache_O              fp32  [P][H][S][D]   (state OUT of partition k)
+ *       cache_L              fp32  [P][H][S]      (state LSE of partition k)
+ *       R (window residual)  fp32  [H][S][D]
+ *     The state of query row s, head h, KV partition k lives at
+ *     cache_O[((k*H + h)*S + s)*D + d] and cache_L[(k*H + h)*S + s].
+ *   - softmax scale is 1/sqrt(D); LSE is a natural logarithm; OUT is
+ *     normalised by the partition's own softmax denominator.
+ */
+#ifndef DT_H_
+#define DT_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DT_API __attribute__((visibility("default")))
+#else
+#define DT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes -------------------------------------------------------- */
+#define DT_OK               0
+#define DT_ERR_INVALID     -1  /* bad argument: shape, null pointer, mode, plan value */
+#define DT_ERR_UNSUPPORTED -2  /* D not in {64, 72, 128}, or a misaligned pointer */
+#define DT_ERR_CACHE_EMPTY -3  /* a REUSE entry names a slot never written (stamp < 0) */
+#define DT_ERR_CUDA        -4  /* a CUDA runtime/driver call failed */
+#define DT_ERR_TIMEOUT     -5  /* (device) a bounded wait inside a kernel ran out */
+
+/* ---- plan modes ---------------------------------------------------------- */
+#define DT_MODE_ALL_COMPUTE 0  /* every pair computed */
+#define DT_MODE_PROXIMITY   1  /* step 1: anchor (all computed); later steps:
+                                  the r partitions farthest from the query's own
+                                  partition are reused, ties to the lower index */
+#define DT_MODE_ALL_REUSE   2  /* every pair reused */
+#define DT_MODE_EXPLICIT    3  /* plan copied from the caller */
+#define DT_MODE_WINDOW      4  /* window + residual: 2 key sets per query tile */
+
+#define DT_PLAN_REUSE   0
+#define DT_PLAN_COMPUTE 1
+
+#define DT_TILE 128             /* query/key tile rows; tiles never straddle a partition */
+
+typedef struct {
+  int32_t H, S, D, P;           /* heads, tokens, head dim, partitions (P ignored in window mode) */
+  int32_t mode;                 /* DT_MODE_* */
+  int32_t reuse_per_row;        /* r: partitions reused per query partition (proximity) */
+  int32_t window;               /* W: key j is in query i's window iff |i-j| <= W/2 (window mode) */
+  int32_t step;                 /* denoising step t, 1-based; step 1 is an anchor */
+} dt_plan_params;
+
+typedef struct {
+  uint8_t* plan;                /* caller-allocated host [nqt][nseg] (out) */
+  int32_t* stamps;              /* caller-allocated host [nqt][nseg] (in/out): step each
+                                   slot was last computed, -1 = never; NULL = all -1 */
+  int64_t computed_blocks;      /* (out) 128x128 blocks whose scores are computed, x H */
+  int64_t skipped_blocks;       /* (out) blocks covered by reused states, x H */
+  int64_t computed_flops;       /* (out) 4*D*(query,key) pairs computed, x H */
+  int32_t nqt;                  /* (out) query tiles per head */
+  int32_t nseg;                 /* (out) key sets per query tile: P, or 2 in window mode */
+} dt_plan;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+DT_API const char* dt_status_string(int status);
+
+/* Number of query tiles per head and of key sets per query tile for these
+ * parameters, so the caller can size dt_plan.plan / dt_plan.stamps.
+ * Query tiles are 128-row, partition-local: nqt = sum_k ceil(|k|/128) with
+ * partition k = [k*c, min((k+1)*c, S)), c = ceil(S/P) ("DiTango", context
+ * partitioning of the sequence).  Host only.  Errors: DT_ERR_INVALID. */
+DT_API int dt_plan_geometry(const dt_plan_params* p, int32_t* nqt, int32_t* nseg);
+
+/* Build the compute/reuse plan of one step on the host ("DiTango", selective
+ * compute and reuse, Fig. 6; anchor steps).  explicit_plan ([nqt][nseg],
+ * values DT_PLAN_*) is read only in DT_MODE_EXPLICIT.  Window mode: key set 0
+ * is the window (always computed), key set 1 its complement, computed at the
+ * anchor step (which makes the residual) and reused afterwards ("DiTFastAttn",
+ * window attention with residual sharing).  Validates that every REUSE entry
+ * has stamp >= 0 (else DT_ERR_CACHE_EMPTY, out->plan left filled, stamps
+ * untouched), then sets stamp = step on COMPUTE entries and fills the counts.
+ * Host only, no CUDA call.  Errors: DT_ERR_INVALID, DT_ERR_CACHE_EMPTY. */
+DT_API int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, dt_plan* out);
+
+/* Fused step on the GPU ("DiTango", attention state Eq. 1-3, composition Eq. 4,
+ * selective reuse Fig. 6).  For each head and query tile and each key set of
+ * the tile's plan row: COMPUTE runs the partial attention (tensor cores) and
+ * writes the fresh state (OUT, LSE) to its cache slot; REUSE reads the cached
+ * state.  All states of the row are composed into O (bf16) and L.
+ *   d_plan      device copy of dt_plan.plan, [nqt][nseg] uint8
+ *   Q, K, V     bf16 [H][S][D] (read)
+ *   cache_O/L   state slots (REUSE slots read, COMPUTE slots written; slots of
+ *               other pairs untouched).  May be NULL in window mode.
+ *   R           window mode only: fp32 [H][S][D]; written at the anchor step
+ *               (R = OUT_full - OUT_window), read afterwards (O = OUT_window + R,
+ *               L = LSE_window).  NULL otherwise.
+ *   O, L        outputs bf16 [H][S][D], fp32 [H][S]
+ *   d_counters  int64[4] device, accumulated (caller zeroes): [0] computed
+ *               blocks and [1] skipped blocks (same definitions as dt_plan),
+ *               [2] fresh states written and [3] cached states read, each
+ *               counted per (query tile, key set, head)
+ *   d_status    int32 device status word (see conventions)
+ * The host validates shapes and alignment before any launch.  One launch. */
+DT_API int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan,
+                          const void* Q, const void* K, const void* V,
+                          float* cache_O, float* cache_L, float* R,
+                          void* O, float* L,
+                          int64_t* d_counters, int32_t* d_status, void* stream);
+
+/* N-way composition of states ("DiTango", composition of attention states,
+ * Eq. 4): for every row, L = M + ln sum_n e^(L_n - M), M = max_n L_n,
+ * OUT = sum_n e^(L_n - L) OUT_n; rows whose N inputs are all empty get
+ * (0, -inf).  O_in fp32 [N][H][S][D], L_in fp32 [N][H][S] (read);
+ * O_out fp32 [H][S][D], L_out fp32 [H][S] (written).  HBM-bound kernel. */
+DT_API int dt_state_merge(int32_t N, int32_t H, int32_t S, int32_t D,
+                   const float* O_in, const float* L_in,
+                   float* O_out, float* L_out, int32_t* d_status, void* stream);
+
+/* Plan-driven scatter of fresh states into the cache ("DiTango", freshly
+ * computed states are stored in the attention state cache): for every
+ * (query tile, partition k) with plan COMPUTE, copy the tile's rows of
+ * fresh_O/fresh_L (layout of cache_O/cache_L) into cache_O/cache_L; REUSE
+ * slots stay byte-identical.  Partition modes only.  HBM-bound kernel. */
+DT_API int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_plan,
+                          const float* fresh_O, const float* fresh_L,
+                          float* cache_O, float* cache_L,
+                          int32_t* d_status, void* stream);
+
+#define DT_WR_MAKE  0   /* R = O_full - O_win                 */
+#define DT_WR_APPLY 1   /* O = bf16(O_win + R)  (O_full unused) */
+
+/* Residual of window attention ("DiTFastAttn", window attention with
+ * residual sharing): MAKE writes R (fp32 [H][S][D]) from O_full and O_win
+ * (fp32 [H][S][D]); APPLY writes O (bf16 [H][S][D]) from O_win and R.
+ * HBM-bound elementwise kernel. */
+DT_API int dt_window_residual(int32_t op, int32_t H, int32_t S, int32_t D,
+                       const float* O_full, const float* O_win,
+                       float* R, void* O, int32_t* d_status, void* stream);
+
+/* Limit, in nanoseconds, of every bounded wait inside the fused kernel
+ * (default 2e9).  A wait that runs out writes DT_ERR_TIMEOUT to *d_status and
+ * the kernel drains its in-flight copies, frees its tensor memory and
+ * returns.  Process-wide setting used by later launches.  Returns DT_OK. */
+DT_API int dt_set_wait_limit_ns(int64_t ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DT_H_ */

@@ -1,0 +1,168 @@
+"""Partitioned attention-state reuse on B200 (sm_100a): Python binding of libdt.
+
+This module only marshals arguments to the C ABI declared in ``include/dt.h``
+(same function names).  Every step of the path runs in libdt: the host plan
+builder and the CUDA kernels.  There is no fallback: if the library is
+missing, every call raises.
+
+Tensors are torch tensors for device memory (``torch.cuda`` streams are passed
+through as raw ``cudaStream_t``); plans and stamps are numpy arrays (host).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+__all__ = [
+    "DtError", "PlanParams", "Plan", "lib_path", "load", "dt_status_string",
+    "dt_plan_geometry", "dt_plan_build", "dt_attn_partial_fused", "dt_state_merge",
+    "dt_state_cache_update", "dt_window_residual", "dt_set_wait_limit_ns",
+    "DT_OK", "DT_ERR_INVALID", "DT_ERR_UNSUPPORTED", "DT_ERR_CACHE_EMPTY", "DT_ERR_CUDA",
+    "DT_ERR_TIMEOUT", "DT_MODE_ALL_COMPUTE", "DT_MODE_PROXIMITY", "DT_MODE_ALL_REUSE",
+    "DT_MODE_EXPLICIT", "DT_MODE_WINDOW", "DT_PLAN_REUSE", "DT_PLAN_COMPUTE", "DT_WR_MAKE",
+    "DT_WR_APPLY", "DT_TILE",
+]
+
+DT_OK, DT_ERR_INVALID, DT_ERR_UNSUPPORTED, DT_ERR_CACHE_EMPTY, DT_ERR_CUDA, DT_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+DT_MODE_ALL_COMPUTE, DT_MODE_PROXIMITY, DT_MODE_ALL_REUSE, DT_MODE_EXPLICIT, DT_MODE_WINDOW = 0, 1, 2, 3, 4
+DT_PLAN_REUSE, DT_PLAN_COMPUTE = 0, 1
+DT_WR_MAKE, DT_WR_APPLY = 0, 1
+DT_TILE = 128
+
+
+class DtError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {dt_status_string(status)} ({status})")
+
+
+class PlanParams(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("S", ctypes.c_int32), ("D", ctypes.c_int32), ("P", ctypes.c_int32),
+                ("mode", ctypes.c_int32), ("reuse_per_row", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("step", ctypes.c_int32)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("plan", ctypes.POINTER(ctypes.c_uint8)), ("stamps", ctypes.POINTER(ctypes.c_int32)),
+                ("computed_blocks", ctypes.c_int64), ("skipped_blocks", ctypes.c_int64),
+                ("computed_flops", ctypes.c_int64), ("nqt", ctypes.c_int32), ("nseg", ctypes.c_int32)]
+
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, "libdt.so")
+
+
+def load() -> ctypes.CDLL:
+    """Load libdt.so from this package directory (raises if it is missing)."""
+    global _LIB
+    if _LIB is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"libdt.so not built ({path}); run python -m partitioned_attention_state_b200.build")
+        lib = ctypes.CDLL(path)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        pp = ctypes.POINTER(PlanParams)
+        sig = {
+            "dt_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "dt_plan_geometry": ([pp, ctypes.POINTER(i32), ctypes.POINTER(i32)], ctypes.c_int),
+            "dt_plan_build": ([pp, vp, ctypes.POINTER(Plan)], ctypes.c_int),
+            "dt_attn_partial_fused": ([pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_state_merge": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_state_cache_update": ([pp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_window_residual": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_set_wait_limit_ns": ([i64], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(lib, name)
+            f.argtypes, f.restype = args, res
+        _LIB = lib
+    return _LIB
+
+
+def _check(status: int, where: str) -> None:
+    if status != DT_OK:
+        raise DtError(status, where)
+
+
+def _ptr(t) -> Optional[int]:
+    """Device/host address of a torch tensor or numpy array (None passes NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def dt_status_string(status: int) -> str:
+    return load().dt_status_string(status).decode()
+
+
+def params(H, S, D, P=1, mode=DT_MODE_ALL_COMPUTE, reuse_per_row=0, window=0, step=1) -> PlanParams:
+    return PlanParams(H, S, D, P, mode, reuse_per_row, window, step)
+
+
+def dt_plan_geometry(p: PlanParams):
+    nqt, nseg = ctypes.c_int32(), ctypes.c_int32()
+    _check(load().dt_plan_geometry(ctypes.byref(p), ctypes.byref(nqt), ctypes.byref(nseg)), "dt_plan_geometry")
+    return nqt.value, nseg.value
+
+
+def dt_plan_build(p: PlanParams, stamps: Optional[np.ndarray] = None, explicit: Optional[np.ndarray] = None):
+    """Host plan of one step.  Returns (plan uint8 [nqt][nseg], counts dict);
+    ``stamps`` (int32 [nqt][nseg]) is updated in place when given."""
+    nqt, nseg = dt_plan_geometry(p)
+    plan = np.zeros((nqt, nseg), dtype=np.uint8)
+    out = Plan()
+    out.plan = plan.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+    if stamps is not None:
+        assert stamps.dtype == np.int32 and stamps.flags.c_contiguous and stamps.size == nqt * nseg
+        out.stamps = stamps.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    ex = None
+    if explicit is not None:
+        ex = np.ascontiguousarray(explicit, dtype=np.uint8)
+    _check(load().dt_plan_build(ctypes.byref(p), _ptr(ex), ctypes.byref(out)), "dt_plan_build")
+    return plan, {"computed_blocks": out.computed_blocks, "skipped_blocks": out.skipped_blocks,
+                  "computed_flops": out.computed_flops}
+
+
+def dt_attn_partial_fused(p: PlanParams, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,
+                          stream=None) -> None:
+    _check(load().dt_attn_partial_fused(ctypes.byref(p), _ptr(d_plan), _ptr(Q), _ptr(K), _ptr(V), _ptr(cache_O),
+                                        _ptr(cache_L), _ptr(R), _ptr(O), _ptr(L), _ptr(d_counters),
+                                        _ptr(d_status), _stream(stream)), "dt_attn_partial_fused")
+
+
+def dt_state_merge(N, H, S, D, O_in, L_in, O_out, L_out, d_status=None, stream=None) -> None:
+    _check(load().dt_state_merge(N, H, S, D, _ptr(O_in), _ptr(L_in), _ptr(O_out), _ptr(L_out), _ptr(d_status),
+                                 _stream(stream)), "dt_state_merge")
+
+
+def dt_state_cache_update(p: PlanParams, d_plan, fresh_O, fresh_L, cache_O, cache_L, d_status=None,
+                          stream=None) -> None:
+    _check(load().dt_state_cache_update(ctypes.byref(p), _ptr(d_plan), _ptr(fresh_O), _ptr(fresh_L),
+                                        _ptr(cache_O), _ptr(cache_L), _ptr(d_status), _stream(stream)),
+           "dt_state_cache_update")
+
+
+def dt_window_residual(op, H, S, D, O_full, O_win, R, O, d_status=None, stream=None) -> None:
+    _check(load().dt_window_residual(op, H, S, D, _ptr(O_full), _ptr(O_win), _ptr(R), _ptr(O), _ptr(d_status),
+                                     _stream(stream)), "dt_window_residual")
+
+
+def dt_set_wait_limit_ns(ns: int) -> None:
+    _check(load().dt_set_wait_limit_ns(int(ns)), "dt_set_wait_limit_ns")

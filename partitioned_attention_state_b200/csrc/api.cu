@@ -1,0 +1,170 @@
+// api.cu -- extern "C" device entry points of libdt: argument validation,
+// TMA descriptor encoding and kernel launches.  No allocation happens here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <cstring>
+
+#include "../../include/dt.h"
+#include "attn_fused.h"
+#include "geometry.h"
+#include "state_ops.h"
+
+namespace {
+
+std::atomic<long long> g_wait_limit_ns{2000000000ll};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count(int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DT_ERR_CUDA;
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) { *out = cached[dev]; return DT_OK; }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return DT_ERR_CUDA;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  *out = n;
+  return DT_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+// bf16 [H][S][D] viewed as a 3-D tensor (D, S, H); box (bw, 128, 1).
+bool encode_qkv(CUtensorMap* m, const void* base, int H, int S, int D, int bw, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
+  cuuint32_t box[3] = {(cuuint32_t)bw, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool shape_ok(int H, int S, int D) {
+  if (H < 0 || S < 0) return false;
+  // int32 row indexing inside the kernels: H*S*D and rows of the cache fit
+  if ((int64_t)H * S * (int64_t)D >= (int64_t)1 << 31) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" int dt_set_wait_limit_ns(int64_t ns) {
+  g_wait_limit_ns.store(ns < 0 ? 0 : ns);
+  return DT_OK;
+}
+
+extern "C" int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan, const void* Q, const void* K,
+                                     const void* V, float* cache_O, float* cache_L, float* R, void* O, float* L,
+                                     int64_t* d_counters, int32_t* d_status, void* stream) {
+  if (!p || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW) return DT_ERR_INVALID;
+  const bool win = p->mode == DT_MODE_WINDOW;
+  if (!shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
+  if (win ? p->window < 1 : p->P < 1) return DT_ERR_INVALID;
+  if (p->D != 64 && p->D != 72 && p->D != 128) return DT_ERR_UNSUPPORTED;
+  if (p->H == 0 || p->S == 0) return DT_OK;
+  if (!d_plan || !Q || !K || !V || !O || !L || !d_status) return DT_ERR_INVALID;
+  if (win ? !R : (!cache_O || !cache_L)) return DT_ERR_INVALID;
+  const void* ptrs[] = {Q, K, V, O, L, d_status};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return DT_ERR_UNSUPPORTED;
+  if ((cache_O && !aligned16(cache_O)) || (cache_L && !aligned16(cache_L)) || (R && !aligned16(R)) ||
+      (d_counters && !aligned16(d_counters)))
+    return DT_ERR_UNSUPPORTED;
+
+  dt::Geom G = dt::make_geom(p->H, p->S, p->D, win ? 1 : p->P, win ? p->window : 0);
+  const int dp = p->D == 72 ? 80 : p->D;
+  dt::AttnParams kp;
+  memset(&kp, 0, sizeof(kp));
+  const CUtensorMapSwizzle sw128 = CU_TENSOR_MAP_SWIZZLE_128B, sw32 = CU_TENSOR_MAP_SWIZZLE_32B;
+  if (!encode_qkv(&kp.tmQ, Q, p->H, p->S, p->D, 64, sw128) || !encode_qkv(&kp.tmK, K, p->H, p->S, p->D, 64, sw128) ||
+      !encode_qkv(&kp.tmV, V, p->H, p->S, p->D, 64, sw128))
+    return DT_ERR_CUDA;
+  if (p->D == 72) {
+    if (!encode_qkv(&kp.tmQt, Q, p->H, p->S, p->D, 16, sw32) || !encode_qkv(&kp.tmKt, K, p->H, p->S, p->D, 16, sw32) ||
+        !encode_qkv(&kp.tmVt, V, p->H, p->S, p->D, 16, sw32))
+      return DT_ERR_CUDA;
+  }
+  kp.plan = d_plan;
+  kp.cache_O = cache_O;
+  kp.cache_L = cache_L;
+  kp.R = R;
+  kp.O = O;
+  kp.L = L;
+  kp.counters = d_counters;
+  kp.status = d_status;
+  kp.H = p->H; kp.S = p->S; kp.D = p->D; kp.P = win ? 1 : p->P; kp.window = win ? p->window : 0;
+  kp.n_items = p->H * G.nqt;
+  kp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->D));
+  kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
+  int sms = 0;
+  if (int e = sm_count(&sms)) return e;
+  int grid = kp.n_items < sms ? kp.n_items : sms;
+  return dt::launch_attn_fused(kp, dp, grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dt_state_merge(int32_t N, int32_t H, int32_t S, int32_t D, const float* O_in, const float* L_in,
+                              float* O_out, float* L_out, int32_t* d_status, void* stream) {
+  if (N < 1 || D < 4 || D % 4 != 0 || !shape_ok(H, S, D)) return DT_ERR_INVALID;
+  if ((int64_t)N * H * S * (int64_t)D >= ((int64_t)1 << 40)) return DT_ERR_INVALID;
+  if ((int64_t)H * S == 0) return DT_OK;
+  if (!O_in || !L_in || !O_out || !L_out) return DT_ERR_INVALID;
+  if (!aligned16(O_in) || !aligned16(O_out) || !aligned16(L_in) || !aligned16(L_out)) return DT_ERR_UNSUPPORTED;
+  (void)d_status;
+  int sms = 0;
+  if (int e = sm_count(&sms)) return e;
+  return dt::launch_state_merge(N, H, S, D, O_in, L_in, O_out, L_out, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_plan, const float* fresh_O,
+                                     const float* fresh_L, float* cache_O, float* cache_L, int32_t* d_status,
+                                     void* stream) {
+  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW)
+    return DT_ERR_INVALID;
+  if (p->P < 1 || p->D < 4 || p->D % 4 != 0 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
+  if (p->H == 0 || p->S == 0) return DT_OK;
+  if (!d_plan || !fresh_O || !fresh_L || !cache_O || !cache_L) return DT_ERR_INVALID;
+  if (!aligned16(fresh_O) || !aligned16(cache_O) || !aligned16(fresh_L) || !aligned16(cache_L))
+    return DT_ERR_UNSUPPORTED;
+  (void)d_status;
+  dt::Geom G = dt::make_geom(p->H, p->S, p->D, p->P, 0);
+  int sms = 0;
+  if (int e = sm_count(&sms)) return e;
+  return dt::launch_cache_update(G, d_plan, fresh_O, fresh_L, cache_O, cache_L, sms,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dt_window_residual(int32_t op, int32_t H, int32_t S, int32_t D, const float* O_full,
+                                  const float* O_win, float* R, void* O, int32_t* d_status, void* stream) {
+  if (op != DT_WR_MAKE && op != DT_WR_APPLY) return DT_ERR_INVALID;
+  if (D < 4 || D % 4 != 0 || !shape_ok(H, S, D)) return DT_ERR_INVALID;
+  const int64_t n = (int64_t)H * S * D;
+  if (n == 0) return DT_OK;
+  if (!O_win || !R || (op == DT_WR_MAKE && !O_full) || (op == DT_WR_APPLY && !O)) return DT_ERR_INVALID;
+  if (!aligned16(O_win) || !aligned16(R) || (O_full && !aligned16(O_full)) || (O && !aligned16(O)))
+    return DT_ERR_UNSUPPORTED;
+  (void)d_status;
+  int sms = 0;
+  if (int e = sm_count(&sms)) return e;
+  return dt::launch_window_residual(op, n, O_full, O_win, R, O, sms, reinterpret_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,608 @@
+// attn_fused_sm100.cu -- fused partial attention with plan-driven state reuse
+// for sm_100a (one persistent kernel; TMA + tcgen05 + TMEM).
+//
+// What it computes ("DiTango: Cost-Effective Parallel Diffusion Generation
+// with Selective Attention State Reuse"):
+//   attention state of query rows over KV partition k (Eq. 1-3):
+//     OUT = softmax(q K_k^T / sqrt(D)) V_k,  LSE = log sum_j exp(q k_j / sqrt(D))
+//   composition of states (Eq. 4), applied over all P partitions of a row;
+//   selective compute/reuse (Fig. 6): per (query tile, partition) the plan says
+//   COMPUTE (fresh state, written to its cache slot) or REUSE (cached state).
+// Window mode ("DiTFastAttn: Attention Compression for Diffusion Transformer
+// Models", window attention with residual sharing): key sets "window" and
+// "complement"; at the anchor step both are computed and R = OUT_full -
+// OUT_window is stored, later steps compute the window only and add R.
+//
+// Work decomposition: a work item is (head, 128-row query tile).  The grid is
+// persistent (one CTA per SM) and strides over items head-major so the CTAs
+// running together share a head's K/V in L2.  Per CTA, 10 warps:
+//   warps 0-3  softmax:   S (TMEM) -> P (bf16, written back over S in TMEM),
+//                         running row max/sum, conditional O rescale
+//   warps 4-7  epilogue:  per computed key set: O_part (TMEM) -> normalised
+//                         fresh state -> cache slot, composed into O_tot (TMEM);
+//                         per reused key set: cached state composed into O_tot;
+//                         per item: O_tot -> O (bf16), LSE
+//   warp 8     MMA:       tcgen05.mma S = Q K^T (smem x smem), O_part += P V
+//                         (P from TMEM, V from smem); TMEM alloc/free
+//   warp 9     TMA:       Q once per item, K/V tiles into an NS-stage ring
+// Tensor memory (512 columns): S/P double buffer [0,256), O_part [256,256+DP),
+// O_tot [256+DP, 256+2*DP).  DP = head dim padded to a multiple of 16 (72 -> 80):
+// a 64-column block uses the 128-byte swizzle, the 16-column tail of D=72 the
+// 32-byte swizzle (zero-filled by TMA out-of-bounds handling).
+//
+// Every wait is bounded; a wait that runs out raises an abort flag shared by
+// all roles, writes DT_ERR_TIMEOUT to *status, and every role drains its
+// in-flight async work before the CTA frees its tensor memory and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dt.h"
+#include "attn_fused.h"
+#include "geometry.h"
+#include "sm100.cuh"
+
+namespace dt {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;
+constexpr uint64_t kDrainLimitNs = 1000000000ull;   // drains use a fixed limit
+__device__ __forceinline__ float neg_inf() { return -__int_as_float(0x7f800000); }
+#define kNegInf (neg_inf())
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
+
+template <int DP>
+struct Cfg {
+  static constexpr int kN64 = DP / 64;                 // 64-column SW128 blocks
+  static constexpr int kTail = (DP % 64) ? 1 : 0;      // one 16-column SW32 block
+  static_assert(DP % 64 == 0 || DP % 64 == 16, "padded head dim must be 64k or 64k+16");
+  static constexpr int kBlk = 128 * 64 * 2;            // bytes of a 128x64 bf16 block
+  static constexpr int kTailBytes = 128 * 16 * 2;      // bytes of a 128x16 bf16 block
+  static constexpr int kTileBytes = kN64 * kBlk + kTail * kTailBytes;   // = 128 * DP * 2
+  static constexpr int kStages = DP == 128 ? 3 : (DP == 80 ? 5 : 6);
+  static constexpr int kColS = 0;
+  static constexpr int kColOpart = 256;
+  static constexpr int kColOtot = 256 + DP;
+  static_assert(kColOtot + DP <= 512, "tensor memory budget");
+  // barrier indices
+  static constexpr int bQFull = 0, bQEmpty = 1, bKFull = 2, bVFull = 2 + kStages, bKVEmpty = 2 + 2 * kStages,
+                       bSFull = 2 + 3 * kStages, bPFull = bSFull + 2, bODone = bPFull + 2, bODSeg = bODone + 1,
+                       bOFree = bODSeg + 1, bStFull = bOFree + 1, bStFree = bStFull + 2, bDrain = bStFree + 2,
+                       kNumBars = bDrain + 1;
+  static constexpr int kStatsBytes = 2 * 2 * 128 * 4;
+  static constexpr int kSmem = kTileBytes * (1 + 2 * kStages) + kStatsBytes + kNumBars * 8 + 16;
+};
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+__device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
+
+// Warp-level wait: lane 0 polls, the verdict is broadcast to the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status,
+                                          uint64_t limit) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status, DT_ERR_TIMEOUT, limit) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool item_has_compute(const Geom& G, int qt, const uint8_t* prow) {
+  for (int s = 0; s < G.P; ++s)
+    if (prow[s] == DT_PLAN_COMPUTE && key_set(G, qt, s).ntiles() > 0) return true;
+  return false;
+}
+
+template <int DP>
+__global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const __grid_constant__ AttnParams p) {
+  using C = Cfg<DP>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {                       // layout needs 1024-byte alignment
+    if (threadIdx.x == 0) atomicCAS(p.status, 0, DT_ERR_UNSUPPORTED);
+    return;
+  }
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + C::kTileBytes;
+  uint8_t* sV = sK + C::kStages * C::kTileBytes;
+  float* stat_m = reinterpret_cast<float*>(sV + C::kStages * C::kTileBytes);   // [2][128]
+  float* stat_l = stat_m + 256;                                                // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stat_l + 256);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Geom G = make_geom(p.H, p.S, p.D, p.P, p.window);
+  const uint64_t lim = p.wait_limit_ns;
+
+  if (warp == 9 && lane == 0) {
+    for (int i = 0; i < C::kNumBars; ++i) mbar_init(&bars[i], 1);
+    mbar_init(&bars[C::bPFull + 0], 4);
+    mbar_init(&bars[C::bPFull + 1], 4);
+    mbar_init(&bars[C::bOFree], 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[C::bStFull + i], 4);
+      mbar_init(&bars[C::bStFree + i], 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&p.tmQ); prefetch_tmap(&p.tmK); prefetch_tmap(&p.tmV);
+      if (C::kTail) { prefetch_tmap(&p.tmQt); prefetch_tmap(&p.tmKt); prefetch_tmap(&p.tmVt); }
+      uint32_t g = 0, nq = 0;
+      for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+        const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
+        const uint8_t* prow = p.plan + (size_t)qt * G.P;
+        if (!item_has_compute(G, qt, prow)) continue;
+        const QTile t = query_tile(G, qt);
+        if (nq > 0 && !mbar_wait(&bars[C::bQEmpty], (nq - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
+          goto tma_done;
+        mbar_arrive_expect_tx(&bars[C::bQFull], C::kTileBytes);
+        for (int c = 0; c < C::kN64; ++c) tma_load_3d(sQ + c * C::kBlk, &p.tmQ, &bars[C::bQFull], 64 * c, t.q0, h);
+        if (C::kTail) tma_load_3d(sQ + C::kN64 * C::kBlk, &p.tmQt, &bars[C::bQFull], 64 * C::kN64, t.q0, h);
+        ++nq;
+        for (int seg = 0; seg < G.P; ++seg) {
+          if (prow[seg] != DT_PLAN_COMPUTE) continue;
+          const KeySet ks = key_set(G, qt, seg);
+          const int nt = ks.ntiles();
+          for (int i = 0; i < nt; ++i, ++g) {
+            const int st = g % C::kStages;
+            if (g >= (uint32_t)C::kStages &&
+                !mbar_wait(&bars[C::bKVEmpty + st], ((g / C::kStages) - 1) & 1, abort_flag, p.status,
+                           DT_ERR_TIMEOUT, lim))
+              goto tma_done;
+            const int row0 = ks.base + ks.tile(i) * kTile;
+            uint8_t* dk = sK + st * C::kTileBytes;
+            uint8_t* dv = sV + st * C::kTileBytes;
+            mbar_arrive_expect_tx(&bars[C::bKFull + st], C::kTileBytes);
+            for (int c = 0; c < C::kN64; ++c) tma_load_3d(dk + c * C::kBlk, &p.tmK, &bars[C::bKFull + st], 64 * c, row0, h);
+            if (C::kTail) tma_load_3d(dk + C::kN64 * C::kBlk, &p.tmKt, &bars[C::bKFull + st], 64 * C::kN64, row0, h);
+            mbar_arrive_expect_tx(&bars[C::bVFull + st], C::kTileBytes);
+            for (int c = 0; c < C::kN64; ++c) tma_load_3d(dv + c * C::kBlk, &p.tmV, &bars[C::bVFull + st], 64 * c, row0, h);
+            if (C::kTail) tma_load_3d(dv + C::kN64 * C::kBlk, &p.tmVt, &bars[C::bVFull + st], 64 * C::kN64, row0, h);
+          }
+        }
+      }
+    tma_done:
+      // let every copy this CTA started land before its shared memory goes away
+      for (int s = 0; s < C::kStages; ++s) {
+        if ((uint32_t)s < g) {
+          const uint32_t last = g - 1 - ((g - 1 - s) % C::kStages);   // latest tile that used stage s
+          const uint32_t ph = (last / C::kStages) & 1;
+          volatile int never = 0;
+          mbar_wait(&bars[C::bKFull + s], ph, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
+          mbar_wait(&bars[C::bVFull + s], ph, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
+        }
+      }
+      if (nq > 0) {
+        volatile int never = 0;
+        mbar_wait(&bars[C::bQFull], (nq - 1) & 1, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64 * C::kN64, 0, 1);
+      constexpr uint32_t idesc_pvt = idesc_bf16_f32(128, 16, 0, 1);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      uint32_t g = 0, nq = 0, cseg = 0;
+      // the PV of the newest tile is issued after the next tile's QK^T
+      int pv_valid = 0, pv_first = 0, pv_last = 0;
+      uint32_t pv_g = 0, pv_seg = 0;
+      bool ok = true;
+
+      auto issue_pv = [&]() -> bool {
+        const uint32_t sb = pv_g & 1;
+        if (!mbar_wait(&bars[C::bPFull + sb], (pv_g >> 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
+          return false;
+        if (pv_first && pv_seg > 0 &&
+            !mbar_wait(&bars[C::bOFree], (pv_seg - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
+          return false;
+        const int st = pv_g % C::kStages;
+        if (!mbar_wait(&bars[C::bVFull + st], (pv_g / C::kStages) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
+          return false;
+        tc_fence_after();
+        const uint32_t aP = tmem + C::kColS + sb * 128;
+        const uint32_t vb = aV + st * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {          // 16 keys per MMA
+          const uint32_t acc = (pv_first && kk == 0) ? 0u : 1u;
+          mma_ts(tmem + C::kColOpart, aP + kk * 8, smem_desc(vb + kk * 2048, C::kBlk, 1024, kSwizzle128B),
+                 idesc_pv, acc);
+          if (C::kTail)
+            mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + kk * 8,
+                   smem_desc(vb + C::kN64 * C::kBlk + kk * 512, C::kTailBytes, 256, kSwizzle32B), idesc_pvt, acc);
+        }
+        mma_commit(&bars[C::bKVEmpty + st]);
+        mma_commit(&bars[C::bODone]);
+        if (pv_last) mma_commit(&bars[C::bODSeg]);
+        return true;
+      };
+
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+        const int qt = idx - (idx / G.nqt) * G.nqt;
+        const uint8_t* prow = p.plan + (size_t)qt * G.P;
+        if (!item_has_compute(G, qt, prow)) continue;
+        if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
+        ++nq;
+        tc_fence_after();
+        for (int seg = 0; seg < G.P && ok; ++seg) {
+          if (prow[seg] != DT_PLAN_COMPUTE) continue;
+          const int nt = key_set(G, qt, seg).ntiles();
+          if (nt == 0) continue;
+          for (int i = 0; i < nt; ++i, ++g) {
+            const int st = g % C::kStages;
+            if (!mbar_wait(&bars[C::bKFull + st], (g / C::kStages) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t dS = tmem + C::kColS + (g & 1) * 128;
+            const uint32_t kb = aK + st * C::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < 4 * C::kN64; ++kk) {      // 16 head-dim columns per MMA
+              const uint32_t off = (kk >> 2) * C::kBlk + (kk & 3) * 32;
+              mma_ss(dS, smem_desc(aQ + off, 16, 1024, kSwizzle128B), smem_desc(kb + off, 16, 1024, kSwizzle128B),
+                     idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            if (C::kTail) {
+              const uint32_t off = C::kN64 * C::kBlk;
+              mma_ss(dS, smem_desc(aQ + off, 16, 256, kSwizzle32B), smem_desc(kb + off, 16, 256, kSwizzle32B),
+                     idesc_qk, 1u);
+            }
+            mma_commit(&bars[C::bSFull + (g & 1)]);
+            if (pv_valid && !issue_pv()) { ok = false; break; }
+            pv_valid = 1; pv_g = g; pv_first = (i == 0); pv_last = (i == nt - 1); pv_seg = cseg;
+          }
+          ++cseg;
+        }
+        mma_commit(&bars[C::bQEmpty]);
+      }
+      if (ok && pv_valid) issue_pv();
+      // all MMAs of this CTA complete before tensor memory is freed
+      mma_commit(&bars[C::bDrain]);
+      volatile int never = 0;
+      mbar_wait(&bars[C::bDrain], 0, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ softmax
+    const int r = warp * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t g = 0, cseg = 0;
+    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+      const int qt = idx - (idx / G.nqt) * G.nqt;
+      const uint8_t* prow = p.plan + (size_t)qt * G.P;
+      if (!item_has_compute(G, qt, prow)) continue;
+      const QTile t = query_tile(G, qt);
+      const int qrow = t.q0 + r;
+      const int q1 = t.q0 + t.rows - 1;
+      for (int seg = 0; seg < G.P; ++seg) {
+        if (prow[seg] != DT_PLAN_COMPUTE) continue;
+        const KeySet ks = key_set(G, qt, seg);
+        const int nt = ks.ntiles();
+        if (nt == 0) continue;
+        float m_run = kNegInf, l_run = 0.f;
+        for (int i = 0; i < nt; ++i, ++g) {
+          const uint32_t sb = g & 1;
+          if (!warp_wait(&bars[C::bSFull + sb], (g >> 1) & 1, abort_flag, p.status, lim)) goto sm_done;
+          tc_fence_after();
+          const int tile = ks.tile(i);
+          const int k0 = ks.base + tile * kTile;
+          const int kvalid = imin(kTile, ks.kend - k0);
+          const uint32_t sc = tmem + lane_base + C::kColS + sb * 128;
+          uint32_t sr[128];
+          tmem_ld32(sc + 0, sr);
+          tmem_ld32(sc + 32, sr + 32);
+          tmem_ld32(sc + 64, sr + 64);
+          tmem_ld32(sc + 96, sr + 96);
+          tmem_wait_ld();
+          int mask_kind = 0;   // 1: keep |i-j| <= hw, 2: keep |i-j| > hw
+          if (G.window > 0)
+            mask_kind = seg == 0 ? (wtile_inside(G, t.q0, q1, tile) ? 0 : 1)
+                                 : (wtile_touches(G, t.q0, q1, tile) ? 2 : 0);
+          if (kvalid < kTile || mask_kind) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+              const int key = k0 + c;
+              const int dist = qrow > key ? qrow - key : key - qrow;
+              bool keep = c < kvalid;
+              if (mask_kind == 1) keep = keep && dist <= G.hw;
+              if (mask_kind == 2) keep = keep && dist > G.hw;
+              if (!keep) sr[c] = f2u(kNegInf);
+            }
+          }
+          float mx = u2f(sr[0]);
+#pragma unroll
+          for (int c = 1; c < 128; ++c) mx = fmaxf(mx, u2f(sr[c]));
+          const float mx2 = mx * sl2;
+          const float m_new = (i == 0) ? mx2 : ((mx2 > m_run + kRescaleThreshold) ? mx2 : m_run);
+          const bool resc = (i > 0) && (m_new != m_run);
+          if (__any_sync(0xffffffffu, resc)) {
+            // O_part holds the previous tiles' sum: wait for its last PV, then rescale
+            if (!warp_wait(&bars[C::bODone], (g - 1) & 1, abort_flag, p.status, lim)) goto sm_done;
+            tc_fence_after();
+            const float alpha = resc ? ex2(m_run - m_new) : 1.f;
+            const uint32_t oc = tmem + lane_base + C::kColOpart;
+#pragma unroll
+            for (int c0 = 0; c0 < DP; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(oc + c0, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) o[j] = f2u(u2f(o[j]) * alpha);
+              tmem_st16(oc + c0, o);
+            }
+            tmem_wait_st();
+            l_run *= alpha;
+          }
+          m_run = m_new;
+          const float m_ref = (m_run == kNegInf) ? 0.f : m_run;
+          float lsum = 0.f;
+          uint32_t pk[64];
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float p0 = ex2(fmaf(u2f(sr[2 * c]), sl2, -m_ref));
+            const float p1 = ex2(fmaf(u2f(sr[2 * c + 1]), sl2, -m_ref));
+            lsum += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          l_run += lsum;
+          tmem_st32(sc + 0, pk);
+          tmem_st32(sc + 32, pk + 32);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[C::bPFull + sb]);
+        }
+        {
+          const uint32_t st = cseg & 1;
+          if (cseg >= 2 && !warp_wait(&bars[C::bStFree + st], ((cseg >> 1) - 1) & 1, abort_flag, p.status, lim))
+            goto sm_done;
+          stat_m[st * 128 + r] = m_run;
+          stat_l[st * 128 + r] = l_run;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[C::bStFull + st]);
+          ++cseg;
+        }
+      }
+    }
+  sm_done:;
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q4 = warp - 4;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t opart = tmem + lane_base + C::kColOpart;
+    const uint32_t otot = tmem + lane_base + C::kColOtot;
+    const int D = p.D;
+    uint32_t cseg = 0;
+    long long n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
+    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+      const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
+      const uint8_t* prow = p.plan + (size_t)qt * G.P;
+      const QTile t = query_tile(G, qt);
+      const int qrow = t.q0 + r;
+      const bool valid = r < t.rows;
+      float m_tot = kNegInf, l_tot = 0.f;
+      bool have = false, use_r = false;
+      for (int seg = 0; seg < G.P; ++seg) {
+        const KeySet ks = key_set(G, qt, seg);
+        const int nt = ks.ntiles();
+        const size_t slot = (((size_t)seg * G.H + h) * G.S + qrow);
+        if (prow[seg] == DT_PLAN_COMPUTE) {
+          if (r == 0) { n_comp += counted_blocks(G, qt, seg); ++n_fresh; }
+          if (nt == 0) {           // empty key set: the identity state
+            if (G.window == 0 && valid) {
+              float4* dst = reinterpret_cast<float4*>(p.cache_O + slot * D);
+              for (int d = 0; d < D / 4; ++d) dst[d] = make_float4(0.f, 0.f, 0.f, 0.f);
+              p.cache_L[slot] = kNegInf;
+            }
+            continue;
+          }
+          const uint32_t st = cseg & 1;
+          if (!warp_wait(&bars[C::bStFull + st], (cseg >> 1) & 1, abort_flag, p.status, lim)) goto ep_done;
+          const float m_s = stat_m[st * 128 + r], l_s = stat_l[st * 128 + r];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[C::bStFree + st]);
+          if (!warp_wait(&bars[C::bODSeg], cseg & 1, abort_flag, p.status, lim)) goto ep_done;
+          tc_fence_after();
+          const bool nonempty = l_s > 0.f;
+          const float inv_l = nonempty ? 1.f / l_s : 0.f;
+          float a, b, m_new;
+          if (!have) { m_new = m_s; a = 0.f; b = nonempty ? 1.f : 0.f; }
+          else {
+            m_new = nonempty ? fmaxf(m_tot, m_s) : m_tot;
+            a = ex2(m_tot - m_new);
+            b = nonempty ? ex2(m_s - m_new) : 0.f;
+          }
+          const float l_new = (have ? a * l_tot : 0.f) + b * l_s;
+          const bool make_r = G.window > 0 && seg == 1;
+          const float inv_tot = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+          const float inv_new = l_new > 0.f ? 1.f / l_new : 0.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < DP; c0 += 16) {
+            uint32_t op[16], ot[16];
+            tmem_ld16(opart + c0, op);
+            tmem_ld16(otot + c0, ot);
+            tmem_wait_ld();
+            float nw[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float x = u2f(op[j]);
+              nw[j] = have ? fmaf(a, u2f(ot[j]), b * x) : b * x;
+            }
+            if (valid) {
+              if (G.window == 0) {
+                float* dst = p.cache_O + slot * D + c0;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                  if (c0 + j < D)
+                    *reinterpret_cast<float4*>(dst + j) =
+                        make_float4(u2f(op[j]) * inv_l, u2f(op[j + 1]) * inv_l, u2f(op[j + 2]) * inv_l,
+                                    u2f(op[j + 3]) * inv_l);
+              } else if (make_r) {
+                float* dst = p.R + ((size_t)h * G.S + qrow) * D + c0;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                  if (c0 + j < D) {
+                    float4 v;
+                    v.x = nw[j] * inv_new - (have ? u2f(ot[j]) * inv_tot : 0.f);
+                    v.y = nw[j + 1] * inv_new - (have ? u2f(ot[j + 1]) * inv_tot : 0.f);
+                    v.z = nw[j + 2] * inv_new - (have ? u2f(ot[j + 2]) * inv_tot : 0.f);
+                    v.w = nw[j + 3] * inv_new - (have ? u2f(ot[j + 3]) * inv_tot : 0.f);
+                    *reinterpret_cast<float4*>(dst + j) = v;
+                  }
+              }
+            }
+            uint32_t o16[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) o16[j] = f2u(nw[j]);
+            tmem_st16(otot + c0, o16);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[C::bOFree]);
+          if (G.window == 0 && valid) p.cache_L[slot] = nonempty ? (m_s + lg2(l_s)) * kLn2 : kNegInf;
+          if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
+          have = have || nonempty;
+          ++cseg;
+        } else {
+          if (r == 0) { n_skip += counted_blocks(G, qt, seg); ++n_read; }
+          if (G.window > 0) { use_r = true; continue; }
+          const float lse_c = valid ? p.cache_L[slot] : kNegInf;
+          const bool nonempty = lse_c > kNegInf;
+          const float m_c = lse_c * kLog2e;
+          float a, b, m_new;
+          if (!have) { m_new = m_c; a = 0.f; b = nonempty ? 1.f : 0.f; }
+          else {
+            m_new = nonempty ? fmaxf(m_tot, m_c) : m_tot;
+            a = ex2(m_tot - m_new);
+            b = nonempty ? ex2(m_c - m_new) : 0.f;
+          }
+          const float l_new = (have ? a * l_tot : 0.f) + b;
+          const float* src = p.cache_O + slot * D;
+#pragma unroll 1
+          for (int c0 = 0; c0 < DP; c0 += 16) {
+            uint32_t ot[16];
+            tmem_ld16(otot + c0, ot);
+            float x[16];
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+              float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (valid && nonempty && c0 + j < D) v = *reinterpret_cast<const float4*>(src + c0 + j);
+              x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
+            }
+            tmem_wait_ld();
+            uint32_t o16[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) o16[j] = f2u(have ? fmaf(a, u2f(ot[j]), b * x[j]) : b * x[j]);
+            tmem_st16(otot + c0, o16);
+          }
+          tmem_wait_st();
+          if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
+          have = have || nonempty;
+        }
+      }
+      // final: O = O_tot / l_tot (+ R), LSE = m_tot + log2(l_tot), in natural units
+      {
+        const float inv = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.O) + ((size_t)h * G.S + qrow) * D;
+        const float* rr = p.R + ((size_t)h * G.S + qrow) * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < DP; c0 += 16) {
+          uint32_t ot[16];
+          tmem_ld16(otot + c0, ot);
+          tmem_wait_ld();
+          if (valid) {
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+              if (c0 + j < D) {
+                float v0 = have ? u2f(ot[j]) * inv : 0.f, v1 = have ? u2f(ot[j + 1]) * inv : 0.f;
+                float v2 = have ? u2f(ot[j + 2]) * inv : 0.f, v3 = have ? u2f(ot[j + 3]) * inv : 0.f;
+                if (use_r) {
+                  const float4 rv = *reinterpret_cast<const float4*>(rr + c0 + j);
+                  v0 += rv.x; v1 += rv.y; v2 += rv.z; v3 += rv.w;
+                }
+                uint2 pk;
+                pk.x = pack_bf16x2(v0, v1);
+                pk.y = pack_bf16x2(v2, v3);
+                *reinterpret_cast<uint2*>(dst + c0 + j) = pk;
+              }
+            }
+          }
+        }
+        if (valid) p.L[(size_t)h * G.S + qrow] = (have && l_tot > 0.f) ? (m_tot + lg2(l_tot)) * kLn2 : kNegInf;
+      }
+    }
+  ep_done:
+    if (r == 0 && p.counters) {
+      atomicAdd(reinterpret_cast<unsigned long long*>(p.counters + 0), (unsigned long long)n_comp);
+      atomicAdd(reinterpret_cast<unsigned long long*>(p.counters + 1), (unsigned long long)n_skip);
+      atomicAdd(reinterpret_cast<unsigned long long*>(p.counters + 2), (unsigned long long)n_fresh);
+      atomicAdd(reinterpret_cast<unsigned long long*>(p.counters + 3), (unsigned long long)n_read);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int DP>
+int launch_dp(const AttnParams& kp, int grid, cudaStream_t stream) {
+  using C = Cfg<DP>;
+  static bool attr_set = false;   // per-process; the attribute is per device function
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(attn_partial_fused_kernel<DP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmem) != cudaSuccess)
+      return DT_ERR_CUDA;
+    attr_set = true;
+  }
+  attn_partial_fused_kernel<DP><<<grid, kThreads, C::kSmem, stream>>>(kp);
+  return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+}
+
+}  // namespace
+
+int attn_fused_smem_bytes(int dp) {
+  switch (dp) {
+    case 64: return Cfg<64>::kSmem;
+    case 80: return Cfg<80>::kSmem;
+    case 128: return Cfg<128>::kSmem;
+  }
+  return -1;
+}
+
+int launch_attn_fused(const AttnParams& kp, int dp, int grid, cudaStream_t stream) {
+  switch (dp) {
+    case 64: return launch_dp<64>(kp, grid, stream);
+    case 80: return launch_dp<80>(kp, grid, stream);
+    case 128: return launch_dp<128>(kp, grid, stream);
+  }
+  return DT_ERR_UNSUPPORTED;
+}
+
+}  // namespace dt

@@ -1,0 +1,157 @@
+// geometry.h -- partition, query-tile and key-tile geometry shared by the host
+// plan builder and the device kernels of libdt.
+//
+// Context partitioning ("DiTango", the sequence is split into P contiguous
+// partitions): c = ceil(S/P), partition k = [k*c, min((k+1)*c, S)).  Query and
+// key tiles are 128 rows and partition-local, so the last tile of a partition
+// may be short and no tile straddles two partitions.
+//
+// Window mode ("DiTFastAttn", window attention): key j is inside query i's
+// window iff |i - j| <= W/2 on the flattened token order; query tiles and key
+// tiles then run over the whole sequence.  A query tile has two key sets:
+//   set 0 "window":     key tiles touching the band, masked to |i-j| <= W/2;
+//   set 1 "complement": every key tile not fully inside the band, masked to
+//                       |i-j| > W/2.
+// Key tiles that straddle the band edge belong to both sets (with opposite
+// masks), so the two sets partition the (query, key) pairs exactly.
+#pragma once
+
+#include <stdint.h>
+
+#if defined(__CUDACC__)
+#define DT_HD __host__ __device__ __forceinline__
+#else
+#define DT_HD inline
+#endif
+
+namespace dt {
+
+constexpr int kTile = 128;
+
+DT_HD int ceil_div(int a, int b) { return (a + b - 1) / b; }
+DT_HD int imin(int a, int b) { return a < b ? a : b; }
+DT_HD int imax(int a, int b) { return a > b ? a : b; }
+
+struct Geom {
+  int H, S, D, P;      // P = number of key sets per query tile (2 in window mode)
+  int window;          // W (window mode) or 0
+  int c;               // partition length (partition modes)
+  int tpp;             // query tiles per full partition (partition modes)
+  int nqt;             // query tiles per head
+  int nkt;             // key tiles over the whole sequence (window mode)
+  int hw;              // W / 2
+};
+
+DT_HD Geom make_geom(int H, int S, int D, int P, int window) {
+  Geom g;
+  g.H = H; g.S = S; g.D = D; g.window = window;
+  g.hw = window / 2;
+  if (window > 0) {
+    g.P = 2;
+    g.c = S;
+    g.tpp = ceil_div(S, kTile);
+    g.nqt = g.tpp;
+    g.nkt = g.tpp;
+  } else {
+    g.P = P;
+    g.c = S > 0 ? ceil_div(S, P) : 0;
+    g.tpp = ceil_div(g.c, kTile);
+    // partitions 0..kl-1 are full (c rows); the last non-empty one may be short
+    int nq = 0;
+    for (int k = 0; k < P; ++k) {
+      int a = imin(k * g.c, S), b = imin((k + 1) * g.c, S);
+      nq += ceil_div(b - a, kTile);
+    }
+    g.nqt = nq;
+    g.nkt = ceil_div(S, kTile);
+  }
+  return g;
+}
+
+DT_HD int part_begin(const Geom& g, int k) { return imin(k * g.c, g.S); }
+DT_HD int part_end(const Geom& g, int k) { return imin((k + 1) * g.c, g.S); }
+
+// Query tile qt -> (partition, first row, rows).
+struct QTile { int part, q0, rows; };
+
+DT_HD QTile query_tile(const Geom& g, int qt) {
+  QTile t;
+  if (g.window > 0) {
+    t.part = 0;
+    t.q0 = qt * kTile;
+    t.rows = imin(kTile, g.S - t.q0);
+  } else {
+    t.part = qt / g.tpp;
+    int j = qt - t.part * g.tpp;
+    t.q0 = part_begin(g, t.part) + j * kTile;
+    t.rows = imin(kTile, part_end(g, t.part) - t.q0);
+  }
+  return t;
+}
+
+// Window-band relations of a query tile [q0, q1] (inclusive) and key tile t.
+DT_HD bool wtile_touches(const Geom& g, int q0, int q1, int t) {
+  int a = t * kTile, b = imin(a + kTile, g.S) - 1;
+  return (a - q1 <= g.hw) && (q0 - b <= g.hw);
+}
+DT_HD bool wtile_inside(const Geom& g, int q0, int q1, int t) {
+  int a = t * kTile, b = imin(a + kTile, g.S) - 1;
+  return (b - q0 <= g.hw) && (q1 - a <= g.hw);
+}
+
+// Key tiles of key set `seg` for query tile `qt`: at most two contiguous
+// ranges of tile indices [r0b, r0e) and [r1b, r1e), tiles indexed relative to
+// `base` (first key row of tile 0 of the set) and clipped to `kend` (one past
+// the set's last key row).
+struct KeySet {
+  int base, kend;
+  int r0b, r0e, r1b, r1e;
+  DT_HD int ntiles() const { return (r0e - r0b) + (r1e - r1b); }
+  // i-th tile of the set (0 <= i < ntiles) -> tile index
+  DT_HD int tile(int i) const { return i < (r0e - r0b) ? r0b + i : r1b + (i - (r0e - r0b)); }
+};
+
+DT_HD KeySet key_set(const Geom& g, int qt, int seg) {
+  KeySet ks;
+  if (g.window == 0) {
+    ks.base = part_begin(g, seg);
+    ks.kend = part_end(g, seg);
+    ks.r0b = 0; ks.r0e = ceil_div(ks.kend - ks.base, kTile);
+    ks.r1b = ks.r1e = 0;
+    return ks;
+  }
+  QTile t = query_tile(g, qt);
+  int q0 = t.q0, q1 = t.q0 + t.rows - 1;
+  ks.base = 0; ks.kend = g.S;
+  // touching range [lo, hi] and fully-inside range [fi, fl] (may be empty)
+  int lo = imax(0, q0 - g.hw) / kTile;
+  int hi = imin(g.S - 1, q1 + g.hw) / kTile;
+  if (seg == 0) {
+    ks.r0b = lo; ks.r0e = hi + 1; ks.r1b = ks.r1e = 0;
+    return ks;
+  }
+  int fi = lo, fl = hi;
+  while (fi <= fl && !wtile_inside(g, q0, q1, fi)) ++fi;
+  while (fl >= fi && !wtile_inside(g, q0, q1, fl)) --fl;
+  if (fi > fl) {            // no tile fully inside: complement spans everything
+    ks.r0b = 0; ks.r0e = g.nkt; ks.r1b = ks.r1e = 0;
+  } else {
+    ks.r0b = 0; ks.r0e = fi; ks.r1b = fl + 1; ks.r1e = g.nkt;
+  }
+  return ks;
+}
+
+// Distinct 128x128 blocks of key set `seg` of query tile `qt` that count as
+// "computed" (or "skipped") blocks: in window mode the straddling tiles are
+// counted once, in the window set.
+DT_HD int counted_blocks(const Geom& g, int qt, int seg) {
+  KeySet ks = key_set(g, qt, seg);
+  if (g.window == 0 || seg == 0) return ks.ntiles();
+  QTile t = query_tile(g, qt);
+  int q0 = t.q0, q1 = t.q0 + t.rows - 1, n = 0;
+  for (int i = 0; i < ks.ntiles(); ++i)
+    if (!wtile_touches(g, q0, q1, ks.tile(i))) ++n;
+  return n;
+}
+
+}  // namespace dt

@@ -1,0 +1,163 @@
+// plan.cpp -- host-side plan builder of libdt (integer work only).
+//
+// "DiTango: Cost-Effective Parallel Diffusion Generation with Selective
+// Attention State Reuse": selective compute and reuse (Fig. 6) -- each query
+// partition computes its own and nearby partitions and reuses cached states of
+// distant ones; spatial locality (Fig. 5a) ranks partitions by distance; anchor
+// steps compute everything.  "DiTFastAttn: Attention Compression for Diffusion
+// Transformer Models" (Approach): window attention with a cached residual is
+// expressed as two key sets per query tile (window, complement).
+#include <cstring>
+#include <vector>
+
+#include "../../include/dt.h"
+#include "geometry.h"
+
+namespace {
+
+bool params_ok(const dt_plan_params* p) {
+  if (!p) return false;
+  if (p->H < 0 || p->S < 0 || p->D < 1 || p->step < 1) return false;
+  if (p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW) return false;
+  if (p->mode == DT_MODE_WINDOW) {
+    if (p->window < 1) return false;
+  } else {
+    if (p->P < 1) return false;
+    if (p->mode == DT_MODE_PROXIMITY && (p->reuse_per_row < 0 || p->reuse_per_row > p->P - 1))
+      return false;
+  }
+  return true;
+}
+
+dt::Geom geom_of(const dt_plan_params* p) {
+  return p->mode == DT_MODE_WINDOW ? dt::make_geom(p->H, p->S, p->D, 1, p->window)
+                                   : dt::make_geom(p->H, p->S, p->D, p->P, 0);
+}
+
+// Proximity row of query partition q: reuse the r partitions farthest from q,
+// equal distances in increasing index order; q itself is never reused.
+void proximity_row(int q, int P, int r, uint8_t* row) {
+  for (int k = 0; k < P; ++k) row[k] = DT_PLAN_COMPUTE;
+  int taken = 0;
+  for (int dist = P - 1; dist >= 1 && taken < r; --dist) {
+    int cand[2] = {q - dist, q + dist};
+    for (int c = 0; c < 2 && taken < r; ++c) {
+      if (cand[c] >= 0 && cand[c] < P) { row[cand[c]] = DT_PLAN_REUSE; ++taken; }
+    }
+  }
+}
+
+int64_t window_pairs(const dt::Geom& g, int q0, int rows) {
+  int64_t n = 0;
+  for (int i = q0; i < q0 + rows; ++i)
+    n += dt::imin(g.S - 1, i + g.hw) - dt::imax(0, i - g.hw) + 1;
+  return n;
+}
+
+}  // namespace
+
+extern "C" const char* dt_status_string(int s) {
+  switch (s) {
+    case DT_OK: return "DT_OK";
+    case DT_ERR_INVALID: return "DT_ERR_INVALID: invalid argument";
+    case DT_ERR_UNSUPPORTED: return "DT_ERR_UNSUPPORTED: unsupported head dim or misaligned pointer";
+    case DT_ERR_CACHE_EMPTY: return "DT_ERR_CACHE_EMPTY: reuse of a cache slot never written";
+    case DT_ERR_CUDA: return "DT_ERR_CUDA: CUDA call failed";
+    case DT_ERR_TIMEOUT: return "DT_ERR_TIMEOUT: a bounded device wait ran out";
+    default: return "unknown dt status";
+  }
+}
+
+extern "C" int dt_plan_geometry(const dt_plan_params* p, int32_t* nqt, int32_t* nseg) {
+  if (!params_ok(p) || !nqt || !nseg) return DT_ERR_INVALID;
+  dt::Geom g = geom_of(p);
+  *nqt = g.nqt;
+  *nseg = g.P;
+  return DT_OK;
+}
+
+extern "C" int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, dt_plan* out) {
+  if (!params_ok(p) || !out || !out->plan) return DT_ERR_INVALID;
+  dt::Geom g = geom_of(p);
+  const int nqt = g.nqt, nseg = g.P;
+  out->nqt = nqt;
+  out->nseg = nseg;
+  out->computed_blocks = out->skipped_blocks = out->computed_flops = 0;
+  const bool anchor = p->step <= 1;
+  uint8_t* plan = out->plan;
+
+  for (int qt = 0; qt < nqt; ++qt) {
+    uint8_t* row = plan + (size_t)qt * nseg;
+    switch (p->mode) {
+      case DT_MODE_ALL_COMPUTE:
+        for (int k = 0; k < nseg; ++k) row[k] = DT_PLAN_COMPUTE;
+        break;
+      case DT_MODE_PROXIMITY:
+        if (anchor) { for (int k = 0; k < nseg; ++k) row[k] = DT_PLAN_COMPUTE; }
+        else proximity_row(dt::query_tile(g, qt).part, nseg, p->reuse_per_row, row);
+        break;
+      case DT_MODE_ALL_REUSE:
+        for (int k = 0; k < nseg; ++k) row[k] = DT_PLAN_REUSE;
+        break;
+      case DT_MODE_EXPLICIT:
+        if (!explicit_plan) return DT_ERR_INVALID;
+        for (int k = 0; k < nseg; ++k) {
+          uint8_t v = explicit_plan[(size_t)qt * nseg + k];
+          if (v != DT_PLAN_COMPUTE && v != DT_PLAN_REUSE) return DT_ERR_INVALID;
+          row[k] = v;
+        }
+        break;
+      case DT_MODE_WINDOW:
+        row[0] = DT_PLAN_COMPUTE;
+        row[1] = anchor ? DT_PLAN_COMPUTE : DT_PLAN_REUSE;
+        break;
+    }
+  }
+
+  // validate reuse against stamps before touching them
+  const size_t n = (size_t)nqt * nseg;
+  for (size_t i = 0; i < n; ++i) {
+    if (plan[i] == DT_PLAN_REUSE) {
+      int32_t s = out->stamps ? out->stamps[i] : -1;
+      if (s < 0) return DT_ERR_CACHE_EMPTY;
+    }
+  }
+  if (out->stamps)
+    for (size_t i = 0; i < n; ++i)
+      if (plan[i] == DT_PLAN_COMPUTE) out->stamps[i] = p->step;
+
+  // counts
+  int64_t cb = 0, sb = 0, fl = 0;
+  const int64_t H = p->H, D = p->D;
+  for (int qt = 0; qt < nqt; ++qt) {
+    const uint8_t* row = plan + (size_t)qt * nseg;
+    dt::QTile t = dt::query_tile(g, qt);
+    if (p->mode == DT_MODE_WINDOW) {
+      int band = dt::counted_blocks(g, qt, 0);
+      int outside = dt::counted_blocks(g, qt, 1);
+      if (row[1] == DT_PLAN_COMPUTE) {
+        cb += H * (band + outside);
+        fl += 4 * H * D * (int64_t)t.rows * g.S;
+      } else {
+        cb += H * band;
+        sb += H * outside;
+        fl += 4 * H * D * window_pairs(g, t.q0, t.rows);
+      }
+    } else {
+      for (int k = 0; k < nseg; ++k) {
+        int len = dt::part_end(g, k) - dt::part_begin(g, k);
+        int64_t nb = H * dt::ceil_div(len, dt::kTile);
+        if (row[k] == DT_PLAN_COMPUTE) {
+          cb += nb;
+          fl += 4 * H * D * (int64_t)t.rows * len;
+        } else {
+          sb += nb;
+        }
+      }
+    }
+  }
+  out->computed_blocks = cb;
+  out->skipped_blocks = sb;
+  out->computed_flops = fl;
+  return DT_OK;
+}

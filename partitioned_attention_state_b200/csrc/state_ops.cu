@@ -1,0 +1,131 @@
+// state_ops.cu -- HBM-bound state kernels of libdt: N-way state composition,
+// plan-driven cache scatter, and the window residual (make / apply).
+//
+// All three stream rows of D fp32 values with 16-byte vector accesses over a
+// flat index, so consecutive threads touch consecutive 16-byte words (fully
+// coalesced); grids are sized in multiples of the SM count.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/dt.h"
+#include "geometry.h"
+#include "state_ops.h"
+
+namespace dt {
+namespace {
+
+constexpr int kBlock = 256;
+__device__ __forceinline__ float neg_inf() { return -__int_as_float(0x7f800000); }
+#define kNegInf (neg_inf())
+
+// "DiTango", composition of attention states (Eq. 4), N-way: per row one max
+// over the N log-sum-exps, then weights e^(L_n - L).
+__global__ void __launch_bounds__(kBlock) state_merge_kernel(int N, int64_t rows, int D, int64_t plane,
+                                                             const float* __restrict__ O_in,
+                                                             const float* __restrict__ L_in,
+                                                             float* __restrict__ O_out, float* __restrict__ L_out) {
+  const int d4n = D / 4;
+  const int64_t total = rows * d4n;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / d4n;
+    const int c4 = (int)(i - row * d4n);
+    float M = kNegInf;
+    for (int n = 0; n < N; ++n) M = fmaxf(M, __ldg(L_in + n * rows + row));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Lr = kNegInf;
+    if (M > kNegInf) {
+      float tot = 0.f;
+      for (int n = 0; n < N; ++n) tot += expf(__ldg(L_in + n * rows + row) - M);
+      Lr = M + logf(tot);
+      for (int n = 0; n < N; ++n) {
+        const float w = expf(__ldg(L_in + n * rows + row) - Lr);
+        const float4 v = __ldg(reinterpret_cast<const float4*>(O_in + n * plane + row * D) + c4);
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+      }
+    }
+    reinterpret_cast<float4*>(O_out + row * D)[c4] = acc;
+    if (c4 == 0) L_out[row] = Lr;
+  }
+}
+
+// "DiTango": freshly computed states are stored in the attention state cache;
+// a slot is written iff its (query tile, partition) entry is COMPUTE.
+__global__ void __launch_bounds__(kBlock) cache_update_kernel(Geom G, const uint8_t* __restrict__ plan,
+                                                              const float* __restrict__ fO,
+                                                              const float* __restrict__ fL, float* __restrict__ cO,
+                                                              float* __restrict__ cL) {
+  const int d4n = G.D / 4;
+  const int64_t rows = (int64_t)G.P * G.H * G.S;
+  const int64_t total = rows * d4n;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / d4n;              // ((k * H + h) * S + s)
+    const int c4 = (int)(i - row * d4n);
+    const int s = (int)(row % G.S);
+    const int k = (int)(row / ((int64_t)G.H * G.S));
+    const int part = s / G.c;
+    const int qt = part * G.tpp + (s - part_begin(G, part)) / kTile;
+    if (plan[(size_t)qt * G.P + k] != DT_PLAN_COMPUTE) continue;
+    reinterpret_cast<float4*>(cO + row * G.D)[c4] = __ldg(reinterpret_cast<const float4*>(fO + row * G.D) + c4);
+    if (c4 == 0) cL[row] = __ldg(fL + row);
+  }
+}
+
+// "DiTFastAttn", window attention with residual sharing.
+__global__ void __launch_bounds__(kBlock) window_residual_kernel(int op, int64_t n4, const float* __restrict__ Of,
+                                                                 const float* __restrict__ Ow, float* __restrict__ R,
+                                                                 __nv_bfloat16* __restrict__ O) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 w = __ldg(reinterpret_cast<const float4*>(Ow) + i);
+    if (op == DT_WR_MAKE) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(Of) + i);
+      reinterpret_cast<float4*>(R)[i] = make_float4(f.x - w.x, f.y - w.y, f.z - w.z, f.w - w.w);
+    } else {
+      const float4 r = __ldg(reinterpret_cast<const float4*>(R) + i);
+      __nv_bfloat162 lo = __floats2bfloat162_rn(w.x + r.x, w.y + r.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(w.z + r.z, w.w + r.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(O)[i] = pk;
+    }
+  }
+}
+
+int grid_for(int64_t work, int sms) {
+  int64_t blocks = (work + kBlock - 1) / kBlock;
+  int64_t cap = (int64_t)sms * 8;           // 8 resident 256-thread blocks per SM
+  if (blocks > cap) blocks = cap;
+  return blocks < 1 ? 1 : (int)blocks;
+}
+
+}  // namespace
+
+int launch_state_merge(int N, int H, int S, int D, const float* O_in, const float* L_in, float* O_out,
+                       float* L_out, int sms, cudaStream_t st) {
+  const int64_t rows = (int64_t)H * S;
+  state_merge_kernel<<<grid_for(rows * (D / 4), sms), kBlock, 0, st>>>(N, rows, D, rows * D, O_in, L_in, O_out,
+                                                                       L_out);
+  return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+}
+
+int launch_cache_update(const Geom& G, const uint8_t* plan, const float* fO, const float* fL, float* cO, float* cL,
+                        int sms, cudaStream_t st) {
+  const int64_t work = (int64_t)G.P * G.H * G.S * (G.D / 4);
+  cache_update_kernel<<<grid_for(work, sms), kBlock, 0, st>>>(G, plan, fO, fL, cO, cL);
+  return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+}
+
+int launch_window_residual(int op, int64_t n, const float* Of, const float* Ow, float* R, void* O, int sms,
+                           cudaStream_t st) {
+  const int64_t n4 = n / 4;
+  window_residual_kernel<<<grid_for(n4, sms), kBlock, 0, st>>>(op, n4, Of, Ow, R,
+                                                              reinterpret_cast<__nv_bfloat16*>(O));
+  return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+}
+
+}  // namespace dt

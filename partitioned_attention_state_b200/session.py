@@ -1,0 +1,92 @@
+"""Device buffers and step sequencing around the libdt C ABI.
+
+A ``Session`` owns the device tensors of one workload (inputs, state cache,
+residual, outputs, counters, status word) and the host stamps, and runs one
+denoising step as: host plan build (``dt_plan_build``) -> plan upload ->
+one fused launch (``dt_attn_partial_fused``).  torch provides the memory and
+the stream; every computation happens in libdt.
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import (DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused, dt_plan_build, dt_plan_geometry, DtError,
+               params)
+
+
+def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
+    """uint16 bf16 bit patterns (host) -> a bf16 tensor on `device`."""
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.to(device).view(torch.bfloat16)
+
+
+class Session:
+    def __init__(self, H: int, S: int, D: int, P: int = 1, mode: int = DT_MODE_PROXIMITY, reuse_per_row: int = 0,
+                 window: int = 0, device: str = "cuda", cache: bool = True):
+        self.H, self.S, self.D, self.P = H, S, D, P
+        self.mode, self.r, self.window = mode, reuse_per_row, window
+        self.device = torch.device(device)
+        win = mode == DT_MODE_WINDOW
+        p = params(H, S, D, P if not win else 1, mode, reuse_per_row, window, 1)
+        self.nqt, self.nseg = dt_plan_geometry(p)
+        dev = self.device
+        self.Q = torch.empty((H, S, D), dtype=torch.bfloat16, device=dev)
+        self.K = torch.empty_like(self.Q)
+        self.V = torch.empty_like(self.Q)
+        self.O = torch.empty_like(self.Q)
+        self.L = torch.empty((H, S), dtype=torch.float32, device=dev)
+        if win:
+            self.cache_O = self.cache_L = None
+            self.R = torch.zeros((H, S, D), dtype=torch.float32, device=dev)
+        else:
+            self.cache_O = torch.zeros((P, H, S, D), dtype=torch.float32, device=dev) if cache else None
+            self.cache_L = torch.full((P, H, S), float("-inf"), dtype=torch.float32, device=dev) if cache else None
+            self.R = None
+        self.d_plan = torch.zeros((max(self.nqt, 1), self.nseg), dtype=torch.uint8, device=dev)
+        self.counters = torch.zeros(4, dtype=torch.int64, device=dev)
+        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.stamps = np.full((self.nqt, self.nseg), -1, dtype=np.int32)
+        self.last_counts = None
+        self.last_plan = None
+
+    # -------------------------------------------------------------- inputs
+    def set_inputs(self, q, k, v) -> None:
+        """q, k, v: uint16 bf16 bit arrays [H][S][D] (host) or bf16 tensors."""
+        for dst, src in ((self.Q, q), (self.K, k), (self.V, v)):
+            if isinstance(src, np.ndarray):
+                dst.copy_(bf16_from_bits(src, "cpu"))
+            else:
+                dst.copy_(src)
+
+    # -------------------------------------------------------------- planning
+    def plan(self, step: int, mode: Optional[int] = None, explicit: Optional[np.ndarray] = None):
+        mode = self.mode if mode is None else mode
+        win = mode == DT_MODE_WINDOW
+        p = params(self.H, self.S, self.D, 1 if win else self.P, mode, self.r, self.window, step)
+        plan, counts = dt_plan_build(p, self.stamps, explicit)
+        return p, plan, counts
+
+    # -------------------------------------------------------------- one step
+    def step(self, step: int, mode: Optional[int] = None, explicit: Optional[np.ndarray] = None,
+             stream=None) -> dict:
+        p, plan, counts = self.plan(step, mode, explicit)
+        if self.nqt > 0:
+            self.d_plan[: self.nqt].copy_(torch.from_numpy(plan))
+        self.launch(p, stream)
+        self.last_counts, self.last_plan = counts, plan
+        return counts
+
+    def launch(self, p, stream=None) -> None:
+        dt_attn_partial_fused(p, self.d_plan, self.Q, self.K, self.V, self.cache_O, self.cache_L, self.R, self.O,
+                              self.L, self.counters, self.status, stream)
+
+    def check(self) -> None:
+        """Synchronise and raise if a kernel reported a device-side error."""
+        torch.cuda.synchronize(self.device)
+        st = int(self.status[0].item())
+        if st != 0:
+            raise DtError(st, "device status")

@@ -1,0 +1,42 @@
+"""Shared helpers of the GPU parity tests: tolerances and comparisons.
+
+Tolerances (bf16 inputs, fp32 accumulation): output O max-abs <= 1e-2 and
+relative RMS <= 5e-3; LSE max-abs <= 1e-3; cached states written this step
+the same; plans, counts and untouched cache slots bit-exact.
+"""
+
+import numpy as np
+
+O_MAX_ABS = 1e-2
+O_REL_RMS = 5e-3
+L_MAX_ABS = 1e-3
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def rel_rms(a, b):
+    den = np.sqrt(np.mean(b * b))
+    return float(np.sqrt(np.mean((a - b) ** 2)) / den) if den > 0 else float(np.sqrt(np.mean(a * a)))
+
+
+def check_out(o_gpu, o_ref, what="O", max_abs=O_MAX_ABS, rel=O_REL_RMS):
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite values"
+    err = np.abs(o_gpu - o_ref)
+    ma, rr = float(err.max()), rel_rms(o_gpu, o_ref)
+    assert ma <= max_abs, f"{what}: max-abs {ma:.3e} > {max_abs}"
+    assert rr <= rel, f"{what}: rel-RMS {rr:.3e} > {rel}"
+    return ma, rr
+
+
+def check_lse(l_gpu, l_ref, what="LSE", max_abs=L_MAX_ABS):
+    l_gpu = np.asarray(l_gpu, dtype=np.float64)
+    neg = ~np.isfinite(l_ref)
+    assert np.array_equal(~np.isfinite(l_gpu), neg), f"{what}: -inf pattern differs"
+    if (~neg).any():
+        ma = float(np.abs(l_gpu[~neg] - l_ref[~neg]).max())
+        assert ma <= max_abs, f"{what}: max-abs {ma:.3e} > {max_abs}"
+        return ma
+    return 0.0

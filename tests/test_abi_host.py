@@ -1,0 +1,155 @@
+"""C-ABI library checks that need no GPU: exports, host plan builder against
+the oracle (bit-exact), status codes and argument validation."""
+
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as orc
+import partitioned_attention_state_b200 as dt
+from partitioned_attention_state_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^DT_API\s+[\w\s\*]+?\b(dt_\w+)\s*\(", text, re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = dt.load()
+    names = header_functions()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for s in (dt.DT_OK, dt.DT_ERR_INVALID, dt.DT_ERR_UNSUPPORTED, dt.DT_ERR_CACHE_EMPTY, dt.DT_ERR_CUDA,
+              dt.DT_ERR_TIMEOUT):
+        assert dt.dt_status_string(s).startswith("DT_")
+    assert "unknown" in dt.dt_status_string(12345)
+
+
+def run_both(mode, H, S, D, P, step, r=0, window=0, stamps=None, explicit=None):
+    p = dt.params(H, S, D, P, mode, r, window, step)
+    st_c = None if stamps is None else stamps.copy()
+    plan_c, counts_c = dt.dt_plan_build(p, st_c, explicit)
+    plan_o, counts_o, st_o = orc.build_plan(mode, H, S, D, P if mode != orc.MODE_WINDOW else 1, step, r=r,
+                                            window=window, stamps=stamps, explicit=explicit)
+    np.testing.assert_array_equal(plan_c, plan_o)
+    assert counts_c == counts_o
+    if st_c is not None:
+        np.testing.assert_array_equal(st_c, st_o)
+    return plan_c, counts_c, st_c
+
+
+@pytest.mark.parametrize("wi", range(len(wl.WORKLOADS)))
+def test_plan_matches_oracle_on_every_workload_schedule(wi):
+    w = wl.WORKLOADS[wi]
+    mode = orc.MODE_WINDOW if w.window else orc.MODE_PROXIMITY
+    for r in w.reuse:
+        p = dt.params(w.H, w.S, w.D, w.P, mode, r, w.window, 1)
+        nqt, nseg = dt.dt_plan_geometry(p)
+        stamps = np.full((nqt, nseg), -1, np.int32)
+        for step in range(1, w.steps + 1):
+            _, _, stamps = run_both(mode, w.H, w.S, w.D, w.P, step, r=r, window=w.window, stamps=stamps)
+
+
+@pytest.mark.parametrize("S,P,r", [(1000, 3, 1), (5, 4, 2), (130, 1, 0), (257, 2, 1), (4097, 7, 5), (300, 5, 4)])
+def test_plan_matches_oracle_ragged_geometry(S, P, r):
+    H, D = 3, 64
+    p = dt.params(H, S, D, P, dt.DT_MODE_PROXIMITY, r, 0, 1)
+    nqt, nseg = dt.dt_plan_geometry(p)
+    assert nqt == len(orc.query_tiles(S, P))
+    st = np.full((nqt, nseg), -1, np.int32)
+    _, _, st = run_both(orc.MODE_PROXIMITY, H, S, D, P, 1, r=r, stamps=st)
+    run_both(orc.MODE_PROXIMITY, H, S, D, P, 2, r=r, stamps=st)
+    run_both(orc.MODE_ALL_REUSE, H, S, D, P, 3, stamps=st)
+    ex = (np.arange(nqt * nseg).reshape(nqt, nseg) % 3 == 0).astype(np.uint8)
+    run_both(orc.MODE_EXPLICIT, H, S, D, P, 3, stamps=st, explicit=ex)
+
+
+@pytest.mark.parametrize("S,W", [(16384, 1024), (1000, 100), (300, 64), (129, 1), (200, 400), (5000, 129)])
+def test_window_plan_matches_oracle(S, W):
+    st = None
+    for step in (1, 2, 3):
+        p = dt.params(2, S, 72, 1, dt.DT_MODE_WINDOW, 0, W, step)
+        nqt, nseg = dt.dt_plan_geometry(p)
+        assert nseg == 2
+        if st is None:
+            st = np.full((nqt, nseg), -1, np.int32)
+        _, _, st = run_both(orc.MODE_WINDOW, 2, S, 72, 1, step, window=W, stamps=st)
+
+
+def test_fig6_row_through_c_abi():
+    p = dt.params(2, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 2, 0, 2)
+    plan, counts = dt.dt_plan_build(p, np.ones((8, 4), np.int32))
+    assert list(plan[0]) == [1, 1, 0, 0]
+    assert (counts["computed_blocks"], counts["skipped_blocks"]) == (64, 64)
+
+
+def test_reuse_without_cache_is_refused_and_stamps_untouched():
+    p = dt.params(2, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 2, 0, 2)
+    st = np.full((8, 4), -1, np.int32)
+    with pytest.raises(dt.DtError) as e:
+        dt.dt_plan_build(p, st)
+    assert e.value.status == dt.DT_ERR_CACHE_EMPTY
+    assert np.all(st == -1)
+    with pytest.raises(dt.DtError):
+        dt.dt_plan_build(dt.params(2, 1024, 64, 4, dt.DT_MODE_ALL_REUSE, 0, 0, 1), None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(P=0), dict(S=-1), dict(step=0), dict(mode=7), dict(r=4), dict(r=-1), dict(mode=4, window=0),
+])
+def test_invalid_plan_params(bad):
+    kw = dict(H=2, S=1024, D=64, P=4, mode=dt.DT_MODE_PROXIMITY, r=1, window=0, step=1)
+    kw.update(bad)
+    p = dt.params(kw["H"], kw["S"], kw["D"], kw["P"], kw["mode"], kw["r"], kw["window"], kw["step"])
+    with pytest.raises(dt.DtError) as e:
+        dt.dt_plan_build(p)
+    assert e.value.status == dt.DT_ERR_INVALID
+
+
+def test_explicit_plan_value_checked():
+    p = dt.params(1, 256, 64, 2, dt.DT_MODE_EXPLICIT, 0, 0, 1)
+    with pytest.raises(dt.DtError):
+        dt.dt_plan_build(p, None, np.full((2, 2), 7, np.uint8))
+
+
+def test_empty_sequence_has_no_tiles():
+    p = dt.params(4, 0, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1)
+    assert dt.dt_plan_geometry(p)[0] == 0
+    plan, counts = dt.dt_plan_build(p)
+    assert plan.size == 0 and counts == {"computed_blocks": 0, "skipped_blocks": 0, "computed_flops": 0}
+
+
+def test_device_entry_points_validate_before_any_cuda_call():
+    """These argument errors are caught on the host, so they run without a GPU."""
+    p = dt.params(2, 1024, 96, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1)
+    lib = dt.load()
+    import ctypes
+    assert lib.dt_attn_partial_fused(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_UNSUPPORTED
+    p.D = 64
+    assert lib.dt_attn_partial_fused(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_INVALID
+    p.H = 0
+    assert lib.dt_attn_partial_fused(ctypes.byref(p), *([None] * 11), None) == dt.DT_OK
+    assert lib.dt_state_merge(0, 1, 1, 64, None, None, None, None, None, None) == dt.DT_ERR_INVALID
+    assert lib.dt_state_merge(2, 1, 1, 66, None, None, None, None, None, None) == dt.DT_ERR_INVALID
+    assert lib.dt_window_residual(5, 1, 1, 64, None, None, None, None, None, None) == dt.DT_ERR_INVALID
+    assert lib.dt_window_residual(0, 1, 8, 64, None, None, None, None, None, None) == dt.DT_ERR_INVALID
+    pw = dt.params(1, 64, 64, 1, dt.DT_MODE_WINDOW, 0, 8, 1)
+    assert lib.dt_state_cache_update(ctypes.byref(pw), *([None] * 7)) == dt.DT_ERR_INVALID
+    # misaligned device pointer is refused on the host
+    p = dt.params(1, 128, 64, 1, dt.DT_MODE_ALL_COMPUTE, 0, 0, 1)
+    fake = [16 * 1024] * 10
+    fake[1] = 16 * 1024 + 2
+    assert lib.dt_attn_partial_fused(ctypes.byref(p), *fake, 16 * 1024, None) == dt.DT_ERR_UNSUPPORTED

@@ -1,0 +1,219 @@
+"""GPU parity: the fused CUDA path against the float64 oracle on the same
+seeded bf16 inputs, through the C ABI.
+
+Small workloads are compared element by element; the full-size ones (in the
+launch configuration the benchmark times) on sampled heads and rows, which
+the oracle follows exactly through the whole schedule (rows are independent).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+import partitioned_attention_state_b200 as dt
+from partitioned_attention_state_b200 import workloads as wl
+from partitioned_attention_state_b200.session import Session
+
+from parity import check_lse, check_out, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dt.dt_set_wait_limit_ns(2_000_000_000)
+    yield
+    torch.cuda.synchronize()
+
+
+def run_partition_schedule(H, S, D, P, schedule, inputs, heads=None, rows=None, check_untouched=False):
+    """schedule: list of (step, mode, r, explicit); inputs: callable -> (q,k,v) bits."""
+    sess = Session(H, S, D, P, mode=dt.DT_MODE_PROXIMITY)
+    cache = orc.StateCache()
+    hs = list(range(H)) if heads is None else list(heads)
+    rs = np.arange(S) if rows is None else np.asarray(rows)
+    for step, mode, r, explicit in schedule:
+        q, k, v = inputs()
+        sess.set_inputs(q, k, v)
+        sess.r = r
+        sess.counters.zero_()
+        before = None
+        if check_untouched:
+            before = (sess.cache_O.clone(), sess.cache_L.clone())
+        counts = sess.step(step, mode=mode, explicit=explicit)
+        sess.check()
+        plan = sess.last_plan
+        # device counters equal the host plan counts (bit-exact)
+        c = sess.counters.cpu().numpy()
+        assert int(c[0]) == counts["computed_blocks"] and int(c[1]) == counts["skipped_blocks"]
+        assert int(c[2]) == H * int((plan == 1).sum()) and int(c[3]) == H * int((plan == 0).sum())
+        Q, K, V = (orc.widen_bf16(x[hs]) for x in (q, k, v))
+        O_ref, L_ref, fresh = orc.partition_step(Q, K, V, plan, S, P, cache, rows=rs)
+        O_gpu = to_np(sess.O[hs][:, rs])
+        L_gpu = to_np(sess.L[hs][:, rs])
+        check_out(O_gpu, O_ref, f"O step {step}")
+        check_lse(L_gpu, L_ref, f"LSE step {step}")
+        # fresh states written to their slots
+        co, cl = sess.cache_O, sess.cache_L
+        for (kk, hi), items in fresh.items():
+            h = hs[hi]
+            for rr, (o_f, l_f) in items:
+                check_out(to_np(co[kk, h][rr]), o_f, f"cache OUT k={kk} h={h} step {step}")
+                check_lse(to_np(cl[kk, h][rr]), l_f, f"cache LSE k={kk} h={h} step {step}")
+        if before is not None:
+            tiles = orc.query_tiles(S, P)
+            for t, (_, q0, q1) in enumerate(tiles):
+                for kk in range(P):
+                    if plan[t, kk] == orc.REUSE:
+                        assert torch.equal(before[0][kk, :, q0:q1], co[kk, :, q0:q1])
+                        assert torch.equal(before[1][kk, :, q0:q1], cl[kk, :, q0:q1])
+    return sess
+
+
+def proximity_schedule(steps, r):
+    return [(t, dt.DT_MODE_PROXIMITY, r, None) for t in range(1, steps + 1)]
+
+
+def stream_of(H, S, D, sigma, seed=0):
+    s = wl.InputStream(H, S, D, sigma, seed=seed)
+    return s.next_step
+
+
+# ----------------------------------------------------------------- workloads
+
+def test_tiny_workload_full_parity():
+    w = wl.WORKLOADS[0]
+    run_partition_schedule(w.H, w.S, w.D, w.P, proximity_schedule(w.steps, w.reuse[0]), wl.stream_for(w).next_step,
+                           check_untouched=True)
+
+
+@pytest.mark.parametrize("r", wl.WORKLOADS[1].reuse)
+def test_dit_xl2_workload_full_parity(r):
+    w = wl.WORKLOADS[1]
+    run_partition_schedule(w.H, w.S, w.D, w.P, proximity_schedule(w.steps, r), wl.stream_for(w).next_step,
+                           check_untouched=True)
+
+
+def sample_rows(S, P, n_extra=40, seed=0):
+    """Rows at tile and partition edges plus random ones."""
+    rows = set()
+    for _, q0, q1 in orc.query_tiles(S, P):
+        rows.update((q0, q1 - 1))
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rows.update(rng.choice(S, size=n_extra, replace=False).tolist())
+    rows = sorted(rows)
+    if len(rows) > 160:
+        keep = set(rng.choice(len(rows), size=160, replace=False).tolist())
+        rows = [r for i, r in enumerate(rows) if i in keep or r in (0, S - 1)]
+    return np.array(sorted(set(rows)))
+
+
+def test_pixart_workload_sampled_rows():
+    w = wl.WORKLOADS[2]
+    run_partition_schedule(w.H, w.S, w.D, w.P, proximity_schedule(2, w.reuse[0]), wl.stream_for(w).next_step,
+                           heads=[0, 7, 15], rows=sample_rows(w.S, w.P))
+
+
+def test_video_workload_full_size_sampled_rows():
+    """Full-size 3D video workload in the benchmark's launch configuration:
+    anchor step, then reuse steps at 25% and 75%."""
+    w = wl.WORKLOADS[3]
+    sched = [(1, dt.DT_MODE_PROXIMITY, 4, None), (2, dt.DT_MODE_PROXIMITY, 4, None),
+             (3, dt.DT_MODE_PROXIMITY, 12, None)]
+    run_partition_schedule(w.H, w.S, w.D, w.P, sched, wl.stream_for(w).next_step, heads=[0, 39],
+                           rows=sample_rows(w.S, w.P, n_extra=24))
+
+
+# ------------------------------------------------------------------ edge cases
+
+@pytest.mark.parametrize("H,S,D,P,r", [
+    (2, 1000, 72, 3, 1),      # ragged partitions and tiles
+    (1, 5, 64, 4, 2),         # tiny sequence, one empty partition
+    (2, 300, 128, 5, 2),      # D=128, short partitions (1 ragged tile each)
+    (3, 2000, 64, 7, 3),
+    (1, 128, 72, 1, 0),       # one tile, one partition
+    (2, 4100, 128, 2, 1),     # 33 key tiles per head, ragged tail of 4 rows
+])
+def test_ragged_geometry(H, S, D, P, r):
+    run_partition_schedule(H, S, D, P, proximity_schedule(3, r), stream_of(H, S, D, 0.05, seed=S),
+                           check_untouched=True)
+
+
+@pytest.mark.parametrize("kind", ["unit", "spiky"])
+@pytest.mark.parametrize("D", [64, 72, 128])
+def test_stress_inputs(kind, D):
+    H, S, P = 2, 700, 3
+    q, k, v = wl.stress_inputs(H, S, D, kind, seed=D)
+    run_partition_schedule(H, S, D, P, [(1, dt.DT_MODE_ALL_COMPUTE, 0, None)], lambda: (q, k, v))
+
+
+def test_all_reuse_reproduces_previous_output_and_explicit_plan():
+    H, S, D, P = 2, 900, 72, 4
+    q, k, v = wl.InputStream(H, S, D, 0.0, seed=5).next_step()
+    sched = [(1, dt.DT_MODE_ALL_COMPUTE, 0, None), (2, dt.DT_MODE_ALL_REUSE, 0, None)]
+    nqt = len(orc.query_tiles(S, P))
+    ex = (np.arange(nqt * P).reshape(nqt, P) % 2).astype(np.uint8)
+    sched.append((3, dt.DT_MODE_EXPLICIT, 0, ex))
+    sess = run_partition_schedule(H, S, D, P, sched, lambda: (q, k, v))
+    # with unchanged inputs every plan gives full attention
+    full, lf = orc.attention_state(orc.widen_bf16(q[1]), orc.widen_bf16(k[1]), orc.widen_bf16(v[1]),
+                                   orc.softmax_scale(D))
+    check_out(to_np(sess.O[1]), full)
+    check_lse(to_np(sess.L[1]), lf)
+
+
+def test_output_guard_bands_untouched():
+    H, S, D, P = 2, 640, 64, 4
+    sess = Session(H, S, D, P, mode=dt.DT_MODE_PROXIMITY)
+    pad = 4096
+    big_o = torch.full((H * S * D + 2 * pad,), 7.0, dtype=torch.bfloat16, device="cuda")
+    big_l = torch.full((H * S + 2 * pad,), 7.0, dtype=torch.float32, device="cuda")
+    sess.O = big_o[pad:pad + H * S * D].view(H, S, D)
+    sess.L = big_l[pad:pad + H * S].view(H, S)
+    sess.set_inputs(*wl.InputStream(H, S, D, 0.05, seed=9).next_step())
+    sess.step(1)
+    sess.check()
+    for t in (big_o[:pad], big_o[-pad:], big_l[:pad], big_l[-pad:]):
+        assert torch.all(t == 7.0)
+    assert torch.isfinite(sess.O.float()).all()
+
+
+# ------------------------------------------------------------------ window mode
+
+def run_window_schedule(H, S, D, W, steps, inputs, heads=None, rows=None):
+    sess = Session(H, S, D, 1, mode=dt.DT_MODE_WINDOW, window=W)
+    R = {}
+    hs = list(range(H)) if heads is None else list(heads)
+    rs = np.arange(S) if rows is None else np.asarray(rows)
+    for step in range(1, steps + 1):
+        q, k, v = inputs()
+        sess.set_inputs(q, k, v)
+        sess.counters.zero_()
+        counts = sess.step(step)
+        sess.check()
+        c = sess.counters.cpu().numpy()
+        assert int(c[0]) == counts["computed_blocks"] and int(c[1]) == counts["skipped_blocks"]
+        Q, K, V = (orc.widen_bf16(x[hs]) for x in (q, k, v))
+        O_ref, L_ref = orc.window_step(Q, K, V, W, step == 1, R, rows=rs)
+        check_out(to_np(sess.O[hs][:, rs]), O_ref, f"O step {step}")
+        check_lse(to_np(sess.L[hs][:, rs]), L_ref, f"LSE step {step}")
+        if step == 1:
+            R_ref = np.stack([np.stack([R[(hi, int(r))] for r in rs]) for hi in range(len(hs))])
+            check_out(to_np(sess.R[hs][:, rs]), R_ref, "R", max_abs=1e-2, rel=1e-2)
+    return sess
+
+
+@pytest.mark.parametrize("H,S,D,W", [(2, 1000, 72, 100), (1, 300, 64, 64), (2, 200, 128, 400), (1, 129, 72, 1),
+                                     (2, 2048, 72, 1024), (1, 5000, 64, 129)])
+def test_window_small(H, S, D, W):
+    run_window_schedule(H, S, D, W, 3, stream_of(H, S, D, 0.03, seed=W))
+
+
+def test_window_workload_full_size_sampled_rows():
+    w = wl.WORKLOADS[4]
+    rows = np.unique(np.concatenate([np.arange(0, 130), np.arange(w.S - 130, w.S),
+                                     np.random.Generator(np.random.PCG64(3)).choice(w.S, 60, replace=False)]))
+    run_window_schedule(w.H, w.S, w.D, w.window, 2, wl.stream_for(w).next_step, heads=[0, 15], rows=rows)
