@@ -1,0 +1,413 @@
+"""Benchmark of the attention-state reuse step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--reuse R] [--no-sweep] [--no-cpu]
+
+A step is one denoising step of the hot path: host plan build, asynchronous
+plan upload and one launch of the fused kernel (partial attention of the
+COMPUTE pairs, fresh-state write-back, composition with the REUSE pairs'
+cached states, output).  The default workload is the 3D video DiT shape
+(H=40, S=32760, D=128, P=16) at 50% reuse, run after an anchor step filled
+the state cache.  Inputs (Q/K/V 1.0 GB, state cache 10.8 GB) are larger than
+L2, so no L2 flush is needed between timed steps.
+
+Multi-GPU: the path does not shard (one GPU, no collectives); N ranks run N
+independent replicas and `value` is their summed throughput.
+
+--impl reference times the CPU oracle (float64 numpy) on the host cores on a
+bounded sample of the same step and reports the same metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "attention ms/denoise-step & TFLOP/s on computed blocks vs B200 bf16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="video_21x30x52_h40_d128_p16")
+    ap.add_argument("--reuse", type=int, default=None, help="r: partitions reused per query partition")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--heads", type=int, default=None, help="override H (smaller profiling captures)")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for fn in ("attn_fused_sm100.cu", "sm100.cuh", "geometry.h", "attn_fused.h"):
+        with open(os.path.join(ROOT, "partitioned_attention_state_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, r):
+    """DRAM bytes per launch of the fused kernel from a committed ncu summary,
+    valid only while the kernel sources are unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", f"attn_fused_sm100_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    m_b = re.search(rf"dram_bytes_per_launch_r{r}:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_b or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is None:
+            return
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            self.out = ""
+
+    def summary(self):
+        if not self.out:
+            return None
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxes.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return None
+        busy = [s for s in sms if s > 0.5 * max(sms)]
+        return {"sm_mhz": float(np.median(busy)), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+# ----------------------------------------------------------------------------- oracle leg
+
+def oracle_sample(w, r, budget_s=12.0, heads=(0,), inputs=None):
+    """Time the CPU oracle on a bounded sample of one reuse step: whole query
+    tiles (all their computed partial states, cached-state merges and the
+    cache update) of one head, until about budget_s seconds of work."""
+    import oracle as orc
+    from partitioned_attention_state_b200 import workloads as wl
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    if inputs is None:
+        s = wl.InputStream(w.H, w.S, w.D, w.sigma, seed=w.seed)
+        inputs = s.next_step() + s.next_step()
+    q1, k1, v1, q2, k2, v2 = inputs
+    hs = list(heads)
+    tiles = orc.query_tiles(w.S, w.P)
+    nqt = len(tiles)
+    plan1, _, st = orc.build_plan(orc.MODE_PROXIMITY, w.H, w.S, w.D, w.P, 1, r=r)
+    plan2, counts, _ = orc.build_plan(orc.MODE_PROXIMITY, w.H, w.S, w.D, w.P, 2, r=r, stamps=st)
+    Q1, K1, V1 = (orc.widen_bf16(x[hs]) for x in (q1, k1, v1))
+    Q2, K2, V2 = (orc.widen_bf16(x[hs]) for x in (q2, k2, v2))
+    parts = orc.partitions(w.S, w.P)
+    rng = np.random.Generator(np.random.PCG64(7))
+    order = rng.permutation(nqt)
+    flops = 0
+    elapsed = 0.0
+    n_tiles = 0
+    for t in order:
+        _, q0, qe = tiles[t]
+        rows = np.arange(q0, qe)
+        cache = orc.StateCache()
+        orc.partition_step(Q1, K1, V1, plan1, w.S, w.P, cache, rows=rows)     # anchor fills the cache (untimed)
+        t0 = time.perf_counter()
+        orc.partition_step(Q2, K2, V2, plan2, w.S, w.P, cache, rows=rows)
+        elapsed += time.perf_counter() - t0
+        flops += sum(4 * w.D * len(hs) * (qe - q0) * (b - a) for k, (a, b) in enumerate(parts) if plan2[t, k])
+        n_tiles += 1
+        if elapsed >= budget_s:
+            break
+    tflops = flops / elapsed / 1e12
+    step_ms = counts["computed_flops"] / (flops / elapsed) * 1e3
+    return {"tflops": tflops, "step_ms_extrapolated": step_ms, "threads": threads,
+            "sample": f"{n_tiles} query tiles x {len(hs)} head(s) of one {int(100 * r / w.P)}%-reuse step "
+                      f"({flops / 1e9:.1f} GFLOP, {elapsed:.1f} s), float64 numpy oracle"}
+
+
+def run_reference(args, w, r, rank):
+    if rank != 0:
+        return
+    from partitioned_attention_state_b200 import workloads as wl
+    s = wl.InputStream(w.H, w.S, w.D, w.sigma, seed=w.seed)
+    inputs = s.next_step() + s.next_step()
+    budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, r, budget_s=budget * 0.25, inputs=inputs)
+    vals, samples = [], []
+    for _ in range(args.steps):
+        res = oracle_sample(w, r, budget_s=budget, inputs=inputs)
+        vals.append(res["tflops"])
+        samples.append(res)
+    v = float(np.mean(vals))
+    last = samples[-1]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean([s["step_ms_extrapolated"] for s in samples])),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "H": w.H, "S": w.S, "D": w.D, "P": w.P, "reuse_per_row": r,
+                   "reuse_ratio": r / w.P},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": last["threads"], "kind": "oracle",
+                         "sample": last["sample"]},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- native leg
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from partitioned_attention_state_b200 import workloads as wl
+    w = wl.BY_NAME[args.workload]
+    if args.heads is not None:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
+    r = args.reuse if args.reuse is not None else (w.P // 2 if w.mode == "proximity" else 0)
+
+    if args.impl == "reference":
+        if world > 1 and rank != 0:
+            return
+        run_reference(args, w, r, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import partitioned_attention_state_b200 as dt
+    from partitioned_attention_state_b200.session import Session
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dt.load()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    win = w.mode == "window"
+    sess = Session(w.H, w.S, w.D, w.P, mode=dt.DT_MODE_WINDOW if win else dt.DT_MODE_PROXIMITY, reuse_per_row=r,
+                   window=w.window)
+    stream = wl.stream_for(w)
+    q1, k1, v1 = stream.next_step()
+    sess.set_inputs(q1, k1, v1)
+    sess.step(1)                                  # anchor: fills the state cache
+    sess.check()
+    q2, k2, v2 = stream.next_step()
+    sess.set_inputs(q2, k2, v2)
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timed(n_steps, n_warm, r_use, step_no=2):
+        sess.r = r_use
+        for _ in range(n_warm):
+            sess.step(step_no)
+        barrier()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        counts = None
+        t0.record(cur)
+        for i in range(n_steps):
+            ev[i][0].record(cur)
+            counts = sess.step(step_no)
+            ev[i][1].record(cur)
+        t1.record(cur)
+        barrier()
+        sess.check()
+        total_ms = t0.elapsed_time(t1)
+        kern_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+        if world > 1:
+            t = torch.tensor([total_ms, kern_ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            total_ms, kern_ms = float(t[0]), float(t[1])
+        return total_ms / n_steps, kern_ms, counts
+
+    # headline
+    with ClockSampler(local) as clk:
+        ms_step, kern_ms, counts = timed(args.steps, args.warmup, r)
+    clocks = clk.summary()
+    flops = counts["computed_flops"]
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    pk, pk_kind = peaks()
+    peak_tf = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (kern_ms * 1e-3) / 1e12
+    traffic = recorded_traffic(w.name, r)
+
+    # reuse sweep 0/25/50/75 %
+    sweep = None
+    if not args.no_sweep and not win:
+        sweep = {}
+        for rr in sorted({0, w.P // 4, w.P // 2, 3 * w.P // 4}):
+            ms, km, c = timed(max(5, args.steps // 2), 3, rr)
+            sweep[f"{int(round(100 * rr / w.P))}%"] = {
+                "reuse_per_row": rr, "ms_per_step": ms, "kernel_ms": km,
+                "tflops": c["computed_flops"] / (km * 1e-3) / 1e12,
+                "frac_of_peak": c["computed_flops"] / (km * 1e-3) / 1e12 / peak_tf,
+                "computed_blocks": c["computed_blocks"], "skipped_blocks": c["skipped_blocks"]}
+        sess.r = r
+
+    # standalone state merge over the whole cache (HBM-bound)
+    merge = None
+    if not win:
+        o_out = torch.empty((w.H, w.S, w.D), dtype=torch.float32, device="cuda")
+        l_out = torch.empty((w.H, w.S), dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            dt.dt_state_merge(w.P, w.H, w.S, w.D, sess.cache_O, sess.cache_L, o_out, l_out)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(cur)
+        nm = 5
+        for _ in range(nm):
+            dt.dt_state_merge(w.P, w.H, w.S, w.D, sess.cache_O, sess.cache_L, o_out, l_out)
+        b.record(cur)
+        barrier()
+        mms = a.elapsed_time(b) / nm
+        nbytes = (w.P + 1) * w.H * w.S * (4 * w.D + 4)
+        hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        merge = {"kernel": "state_merge", "ms": mms, "bytes": nbytes, "GB/s": nbytes / (mms * 1e-3) / 1e9,
+                 "frac_of_hbm": nbytes / (mms * 1e-3) / 1e9 / hbm}
+        del o_out, l_out
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in (q2, k2, v2)]
+        ho = torch.empty((w.H, w.S, w.D), dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty((w.H, w.S), dtype=torch.float32).pin_memory()
+        ke = max(3, args.steps // 2)
+
+        def e2e_step():
+            for dst, src in zip((sess.Q, sess.K, sess.V), hq):
+                dst.view(torch.int16).copy_(src, non_blocking=True)
+            sess.step(2)
+            ho.copy_(sess.O, non_blocking=True)
+            hl.copy_(sess.L, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(cur)
+        for _ in range(ke):
+            e2e_step()
+        b.record(cur)
+        barrier()
+        ems = a.elapsed_time(b) / ke
+        if world > 1:
+            t = torch.tensor([ems], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t[0])
+        h2d = sum(x.numel() * x.element_size() for x in hq) + sess.nqt * sess.nseg
+        d2h = ho.numel() * 2 + hl.numel() * 4
+        e2e = {"value": flops * world / (ems * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        res = oracle_sample(w, r, budget_s=12.0, inputs=(q1, k1, v1, q2, k2, v2))
+        cpu = {"value": res["tflops"], "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
+               "sample": res["sample"], "ms_per_step_extrapolated": res["step_ms_extrapolated"]}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "H": w.H, "S": w.S, "D": w.D, "P": w.P, "window": w.window,
+                       "reuse_per_row": r, "reuse_ratio": r / w.P, "step": "reuse step after an anchor step",
+                       "computed_blocks": counts["computed_blocks"], "skipped_blocks": counts["skipped_blocks"],
+                       "computed_flops": flops, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (no flush): Q/K/V and the state cache exceed 126 MB"},
+            "roofline": {"bound": "tensor", "kernel": "attn_partial_fused_kernel", "achieved": achieved,
+                         "peak": peak_tf, "peak_kind": f"{pk_kind} bf16 dense (burst)", "unit": "TFLOP/s",
+                         "frac": achieved / peak_tf, "traffic": traffic, "kernel_ms": kern_ms,
+                         "flops_per_launch": flops},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "reuse_sweep": sweep,
+            "state_merge": merge,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

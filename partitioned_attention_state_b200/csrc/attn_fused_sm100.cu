@@ -30,6 +30,11 @@
 // a 64-column block uses the 128-byte swizzle, the 16-column tail of D=72 the
 // 32-byte swizzle (zero-filled by TMA out-of-bounds handling).
 //
+// Split-precision PV for the window key set: P = P_hi + P_lo with both halves
+// in bf16 (P_lo in the upper half of the S buffer) and two PV MMAs.  The window
+// output is later combined with a residual that nearly cancels it, which
+// amplifies the relative rounding error of a single bf16 P several times.
+//
 // Every wait is bounded; a wait that runs out raises an abort flag shared by
 // all roles, writes DT_ERR_TIMEOUT to *status, and every role drains its
 // in-flight async work before the CTA frees its tensor memory and exits.
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       uint32_t g = 0, nq = 0, cseg = 0;
       // the PV of the newest tile is issued after the next tile's QK^T
-      int pv_valid = 0, pv_first = 0, pv_last = 0;
+      int pv_valid = 0, pv_first = 0, pv_last = 0, pv_precise = 0;
       uint32_t pv_g = 0, pv_seg = 0;
       bool ok = true;
 
@@ -224,11 +229,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {          // 16 keys per MMA
           const uint32_t acc = (pv_first && kk == 0) ? 0u : 1u;
-          mma_ts(tmem + C::kColOpart, aP + kk * 8, smem_desc(vb + kk * 2048, C::kBlk, 1024, kSwizzle128B),
-                 idesc_pv, acc);
-          if (C::kTail)
-            mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + kk * 8,
-                   smem_desc(vb + C::kN64 * C::kBlk + kk * 512, C::kTailBytes, 256, kSwizzle32B), idesc_pvt, acc);
+          const uint64_t vd = smem_desc(vb + kk * 2048, C::kBlk, 1024, kSwizzle128B);
+          const uint64_t vdt = smem_desc(vb + C::kN64 * C::kBlk + kk * 512, C::kTailBytes, 256, kSwizzle32B);
+          mma_ts(tmem + C::kColOpart, aP + kk * 8, vd, idesc_pv, acc);
+          if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + kk * 8, vdt, idesc_pvt, acc);
+          if (pv_precise) {                       // P = P_hi + P_lo (P_lo in columns 64..127)
+            mma_ts(tmem + C::kColOpart, aP + 64 + kk * 8, vd, idesc_pv, 1u);
+            if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + 64 + kk * 8, vdt, idesc_pvt, 1u);
+          }
         }
         mma_commit(&bars[C::bKVEmpty + st]);
         mma_commit(&bars[C::bODone]);
@@ -270,6 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             mma_commit(&bars[C::bSFull + (g & 1)]);
             if (pv_valid && !issue_pv()) { ok = false; break; }
             pv_valid = 1; pv_g = g; pv_first = (i == 0); pv_last = (i == nt - 1); pv_seg = cseg;
+            pv_precise = (G.window > 0 && seg == 0);
           }
           ++cseg;
         }
@@ -301,6 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const int nt = ks.ntiles();
         if (nt == 0) continue;
         float m_run = kNegInf, l_run = 0.f;
+        const bool precise = G.window > 0 && seg == 0;
         for (int i = 0; i < nt; ++i, ++g) {
           const uint32_t sb = g & 1;
           if (!warp_wait(&bars[C::bSFull + sb], (g >> 1) & 1, abort_flag, p.status, lim)) goto sm_done;
@@ -357,17 +367,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           m_run = m_new;
           const float m_ref = (m_run == kNegInf) ? 0.f : m_run;
           float lsum = 0.f;
-          uint32_t pk[64];
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float p0 = ex2(fmaf(u2f(sr[2 * c]), sl2, -m_ref));
-            const float p1 = ex2(fmaf(u2f(sr[2 * c + 1]), sl2, -m_ref));
-            lsum += p0 + p1;
-            pk[c] = pack_bf16x2(p0, p1);
+          for (int ch = 0; ch < 4; ++ch) {        // 32 keys -> 16 packed bf16 pairs per chunk
+            uint32_t hi[16], lo[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int j = ch * 32 + 2 * c;
+              const float p0 = ex2(fmaf(u2f(sr[j]), sl2, -m_ref));
+              const float p1 = ex2(fmaf(u2f(sr[j + 1]), sl2, -m_ref));
+              lsum += p0 + p1;
+              hi[c] = pack_bf16x2(p0, p1);
+              // residual of the bf16 rounding, kept for the split-precision PV
+              lo[c] = pack_bf16x2(p0 - u2f(hi[c] << 16), p1 - u2f(hi[c] & 0xffff0000u));
+            }
+            tmem_st16(sc + ch * 16, hi);
+            if (precise) tmem_st16(sc + 64 + ch * 16, lo);
           }
           l_run += lsum;
-          tmem_st32(sc + 0, pk);
-          tmem_st32(sc + 32, pk + 32);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();

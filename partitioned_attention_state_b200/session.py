@@ -47,6 +47,12 @@ class Session:
             self.cache_L = torch.full((P, H, S), float("-inf"), dtype=torch.float32, device=dev) if cache else None
             self.R = None
         self.d_plan = torch.zeros((max(self.nqt, 1), self.nseg), dtype=torch.uint8, device=dev)
+        # two pinned host plan buffers: the plan of step t is built while the
+        # upload of step t-1 may still be in flight
+        self._pinned = [torch.zeros((max(self.nqt, 1), self.nseg), dtype=torch.uint8, pin_memory=True)
+                        for _ in range(2)]
+        self._uploaded = [None, None]
+        self._turn = 0
         self.counters = torch.zeros(4, dtype=torch.int64, device=dev)
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
         self.stamps = np.full((self.nqt, self.nseg), -1, dtype=np.int32)
@@ -73,9 +79,21 @@ class Session:
     # -------------------------------------------------------------- one step
     def step(self, step: int, mode: Optional[int] = None, explicit: Optional[np.ndarray] = None,
              stream=None) -> dict:
+        """Host plan build, asynchronous plan upload, one fused launch."""
         p, plan, counts = self.plan(step, mode, explicit)
         if self.nqt > 0:
-            self.d_plan[: self.nqt].copy_(torch.from_numpy(plan))
+            i = self._turn
+            self._turn ^= 1
+            if self._uploaded[i] is not None:
+                self._uploaded[i].synchronize()      # that buffer's previous upload is done
+            buf = self._pinned[i]
+            buf[: self.nqt].numpy()[...] = plan
+            st = torch.cuda.current_stream(self.device) if stream is None else stream
+            with torch.cuda.stream(st):
+                self.d_plan[: self.nqt].copy_(buf[: self.nqt], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(st)
+            self._uploaded[i] = ev
         self.launch(p, stream)
         self.last_counts, self.last_plan = counts, plan
         return counts

@@ -21,12 +21,19 @@ def rel_rms(a, b):
     return float(np.sqrt(np.mean((a - b) ** 2)) / den) if den > 0 else float(np.sqrt(np.mean(a * a)))
 
 
-def check_out(o_gpu, o_ref, what="O", max_abs=O_MAX_ABS, rel=O_REL_RMS):
+BF16_QUANTUM = 2.0 ** -8     # relative spacing of bf16 values at the bottom of a binade
+
+
+def check_out(o_gpu, o_ref, what="O", max_abs=O_MAX_ABS, rel=O_REL_RMS, output_scaled=False):
+    """max-abs and relative-RMS check.  ``output_scaled`` (unit-variance
+    stress inputs only, where |O| reaches 4 and a bf16 output's own rounding
+    exceeds 1e-2) widens the max-abs bound by one bf16 quantum of |O_ref|."""
     o_gpu = np.asarray(o_gpu, dtype=np.float64)
     assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite values"
     err = np.abs(o_gpu - o_ref)
+    bound = max_abs + (BF16_QUANTUM * np.abs(o_ref) if output_scaled else 0.0)
     ma, rr = float(err.max()), rel_rms(o_gpu, o_ref)
-    assert ma <= max_abs, f"{what}: max-abs {ma:.3e} > {max_abs}"
+    assert np.all(err <= bound), f"{what}: max-abs {ma:.3e} > {max_abs} (+bf16 quantum: {output_scaled})"
     assert rr <= rel, f"{what}: rel-RMS {rr:.3e} > {rel}"
     return ma, rr
 
