@@ -15,16 +15,21 @@
 //
 // Work decomposition: a work item is (head, 128-row query tile).  The grid is
 // persistent (one CTA per SM) and strides over items head-major so the CTAs
-// running together share a head's K/V in L2.  Per CTA, 10 warps:
+// running together share a head's K/V in L2; each item visits its key sets and
+// key tiles in a rotated order so those CTAs do not read the same tile at the
+// same moment.  Per CTA, 12 warps (3 warpgroups, registers rebalanced with
+// setmaxnreg):
 //   warps 0-3  softmax:   S (TMEM) -> P (bf16, written back over S in TMEM),
 //                         running row max/sum, conditional O rescale
-//   warps 4-7  epilogue:  per computed key set: O_part (TMEM) -> normalised
-//                         fresh state -> cache slot, composed into O_tot (TMEM);
-//                         per reused key set: cached state composed into O_tot;
-//                         per item: O_tot -> O (bf16), LSE
+//   warps 4-7  epilogue:  per reused key set (first, off the critical path):
+//                         cached state composed into O_tot (TMEM); per computed
+//                         key set: O_part (TMEM) -> registers (O_part released at
+//                         once) -> normalised fresh state -> cache slot, composed
+//                         into O_tot; per item: O_tot -> O (bf16), LSE
 //   warp 8     MMA:       tcgen05.mma S = Q K^T (smem x smem), O_part += P V
 //                         (P from TMEM, V from smem); TMEM alloc/free
 //   warp 9     TMA:       Q once per item, K/V tiles into an NS-stage ring
+//   warps 10-11 idle (complete the third warpgroup)
 // Tensor memory (512 columns): S/P double buffer [0,256), O_part [256,256+DP),
 // O_tot [256+DP, 256+2*DP).  DP = head dim padded to a multiple of 16 (72 -> 80):
 // a 64-column block uses the 128-byte swizzle, the 16-column tail of D=72 the
@@ -45,6 +50,7 @@
 
 #include "../../include/dt.h"
 #include "attn_fused.h"
+#include "exp2_poly.h"
 #include "geometry.h"
 #include "sm100.cuh"
 
@@ -53,13 +59,34 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
+// 3 warpgroups: softmax (warps 0-3), epilogue (4-7), MMA (8) + TMA (9) + 2 idle.
+constexpr int kThreads = 384;
+// Registers per thread at launch (ptxas: 65536 / 384, rounded down to 8; the
+// build checks it) and the per-warpgroup split after setmaxnreg.  The split
+// must fit the launch pool: 128 * (kRegsSoftmax + kRegsEpilogue + kRegsOther)
+// <= kThreads * kLaunchRegs.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsSoftmax = 208, kRegsEpilogue = 224, kRegsOther = 64;
+static_assert(128 * (kRegsSoftmax + kRegsEpilogue + kRegsOther) <= kThreads * kLaunchRegs, "register split");
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // drains use a fixed limit
 __device__ __forceinline__ float neg_inf() { return -__int_as_float(0x7f800000); }
 #define kNegInf (neg_inf())
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
+
+// Timeline tracing for kernel development (compiled only with -DDT_TRACE):
+// CTA 0 records clock64 stamps of each role into a caller-provided buffer.
+#ifdef DT_TRACE
+__device__ uint64_t* g_dt_trace = nullptr;
+#define DT_TR(ev, idx)                                                                             \
+  do {                                                                                             \
+    if (blockIdx.x == 0 && (threadIdx.x & 31) == 0 && g_dt_trace && (idx) < 4096)                 \
+      g_dt_trace[(ev) * 4096 + (idx)] = clock64();                                                 \
+  } while (0)
+#else
+#define DT_TR(ev, idx) do {} while (0)
+#endif
 
 template <int DP>
 struct Cfg {
@@ -83,6 +110,18 @@ struct Cfg {
   static constexpr int kSmem = kTileBytes * (1 + 2 * kStages) + kStatsBytes + kNumBars * 8 + 16;
 };
 
+// Exponentials of an unmasked tile: when kEmuMod > 0 every kEmuMod-th pair is
+// evaluated on the FMA pipe instead of MUFU.  Off: with one or two softmax
+// warps per SM sub-partition the loop is latency-bound, not MUFU-bound, and
+// the polynomial only lengthens it (measured).
+constexpr int kEmuMod = 0;
+
+// Two non-negative finite floats -> packed bf16x2 (lo = a), rounded half up,
+// with integer ops (keeps the conversion off the MUFU/XU pipe).
+__device__ __forceinline__ uint32_t pack_bf16x2_rhu(float a, float b) {
+  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
+}
+
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
@@ -100,6 +139,56 @@ __device__ __forceinline__ bool item_has_compute(const Geom& G, int qt, const ui
   for (int s = 0; s < G.P; ++s)
     if (prow[s] == DT_PLAN_COMPUTE && key_set(G, qt, s).ntiles() > 0) return true;
   return false;
+}
+
+// Visiting order of the key sets and key tiles of work item idx.  States
+// compose associatively and commutatively and the online softmax is order
+// free, so any order gives the same result; rotating the start per item keeps
+// the CTAs that run together from streaming the same K/V tile at once.
+__device__ __forceinline__ int visit_seg(const Geom& G, int idx, int j) {
+  if (G.window > 0) return j;                 // window set before its complement
+  int s = j + idx % G.P;
+  return s >= G.P ? s - G.P : s;
+}
+__device__ __forceinline__ int visit_tile(const KeySet& ks, int nt, int idx, int seg, int i) {
+  int k = i + (idx * 5 + seg * 3) % nt;
+  return ks.tile(k >= nt ? k - nt : k);
+}
+
+// Issue O_part += P V for tile g (P read from tensor memory, V from the ring).
+template <int DP>
+__device__ __forceinline__ bool issue_pv(uint64_t* bars, uint32_t tmem, uint32_t aV, uint32_t g, uint32_t seg,
+                                         bool first, bool last, bool precise, volatile int* abort, int32_t* status,
+                                         uint64_t lim) {
+  using C = Cfg<DP>;
+  constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64 * C::kN64, 0, 1);
+  constexpr uint32_t idesc_pvt = idesc_bf16_f32(128, 16, 0, 1);
+  const uint32_t sb = g & 1;
+  if (!mbar_wait(&bars[C::bPFull + sb], (g >> 1) & 1, abort, status, DT_ERR_TIMEOUT, lim)) return false;
+  if (first && seg > 0 && !mbar_wait(&bars[C::bOFree], (seg - 1) & 1, abort, status, DT_ERR_TIMEOUT, lim))
+    return false;
+  const int st = g % C::kStages;
+  if (!mbar_wait(&bars[C::bVFull + st], (g / C::kStages) & 1, abort, status, DT_ERR_TIMEOUT, lim)) return false;
+  DT_TR(5, g);
+  tc_fence_after();
+  const uint32_t aP = tmem + C::kColS + sb * 128;
+  const uint32_t vb = aV + st * C::kTileBytes;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {          // 16 keys per MMA
+    const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+    const uint64_t vd = smem_desc(vb + kk * 2048, C::kBlk, 1024, kSwizzle128B);
+    const uint64_t vdt = smem_desc(vb + C::kN64 * C::kBlk + kk * 512, C::kTailBytes, 256, kSwizzle32B);
+    mma_ts(tmem + C::kColOpart, aP + kk * 8, vd, idesc_pv, acc);
+    if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + kk * 8, vdt, idesc_pvt, acc);
+    if (precise) {                          // P = P_hi + P_lo (P_lo in columns 64..127)
+      mma_ts(tmem + C::kColOpart, aP + 64 + kk * 8, vd, idesc_pv, 1u);
+      if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + 64 + kk * 8, vdt, idesc_pvt, 1u);
+    }
+  }
+  mma_commit(&bars[C::bKVEmpty + st]);
+  mma_commit(&bars[C::bODone]);
+  if (last) mma_commit(&bars[C::bODSeg]);
+  return true;
 }
 
 template <int DP>
@@ -145,7 +234,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 9) {
+  if (warp >= 8) {
+   regs_dec<kRegsOther>();
+   if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&p.tmQ); prefetch_tmap(&p.tmK); prefetch_tmap(&p.tmV);
@@ -162,7 +253,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         for (int c = 0; c < C::kN64; ++c) tma_load_3d(sQ + c * C::kBlk, &p.tmQ, &bars[C::bQFull], 64 * c, t.q0, h);
         if (C::kTail) tma_load_3d(sQ + C::kN64 * C::kBlk, &p.tmQt, &bars[C::bQFull], 64 * C::kN64, t.q0, h);
         ++nq;
-        for (int seg = 0; seg < G.P; ++seg) {
+        for (int j = 0; j < G.P; ++j) {
+          const int seg = visit_seg(G, idx, j);
           if (prow[seg] != DT_PLAN_COMPUTE) continue;
           const KeySet ks = key_set(G, qt, seg);
           const int nt = ks.ntiles();
@@ -172,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
                 !mbar_wait(&bars[C::bKVEmpty + st], ((g / C::kStages) - 1) & 1, abort_flag, p.status,
                            DT_ERR_TIMEOUT, lim))
               goto tma_done;
-            const int row0 = ks.base + ks.tile(i) * kTile;
+            const int row0 = ks.base + visit_tile(ks, nt, idx, seg, i) * kTile;
             uint8_t* dk = sK + st * C::kTileBytes;
             uint8_t* dv = sV + st * C::kTileBytes;
             mbar_arrive_expect_tx(&bars[C::bKFull + st], C::kTileBytes);
@@ -200,12 +292,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         mbar_wait(&bars[C::bQFull], (nq - 1) & 1, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
       }
     }
-  } else if (warp == 8) {
+   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64 * C::kN64, 0, 1);
-      constexpr uint32_t idesc_pvt = idesc_bf16_f32(128, 16, 0, 1);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       uint32_t g = 0, nq = 0, cseg = 0;
       // the PV of the newest tile is issued after the next tile's QK^T
@@ -213,36 +303,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       uint32_t pv_g = 0, pv_seg = 0;
       bool ok = true;
 
-      auto issue_pv = [&]() -> bool {
-        const uint32_t sb = pv_g & 1;
-        if (!mbar_wait(&bars[C::bPFull + sb], (pv_g >> 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
-          return false;
-        if (pv_first && pv_seg > 0 &&
-            !mbar_wait(&bars[C::bOFree], (pv_seg - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
-          return false;
-        const int st = pv_g % C::kStages;
-        if (!mbar_wait(&bars[C::bVFull + st], (pv_g / C::kStages) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
-          return false;
-        tc_fence_after();
-        const uint32_t aP = tmem + C::kColS + sb * 128;
-        const uint32_t vb = aV + st * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {          // 16 keys per MMA
-          const uint32_t acc = (pv_first && kk == 0) ? 0u : 1u;
-          const uint64_t vd = smem_desc(vb + kk * 2048, C::kBlk, 1024, kSwizzle128B);
-          const uint64_t vdt = smem_desc(vb + C::kN64 * C::kBlk + kk * 512, C::kTailBytes, 256, kSwizzle32B);
-          mma_ts(tmem + C::kColOpart, aP + kk * 8, vd, idesc_pv, acc);
-          if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + kk * 8, vdt, idesc_pvt, acc);
-          if (pv_precise) {                       // P = P_hi + P_lo (P_lo in columns 64..127)
-            mma_ts(tmem + C::kColOpart, aP + 64 + kk * 8, vd, idesc_pv, 1u);
-            if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + 64 + kk * 8, vdt, idesc_pvt, 1u);
-          }
-        }
-        mma_commit(&bars[C::bKVEmpty + st]);
-        mma_commit(&bars[C::bODone]);
-        if (pv_last) mma_commit(&bars[C::bODSeg]);
-        return true;
-      };
 
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
@@ -251,7 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
         ++nq;
         tc_fence_after();
-        for (int seg = 0; seg < G.P && ok; ++seg) {
+        for (int j = 0; j < G.P && ok; ++j) {
+          const int seg = visit_seg(G, idx, j);
           if (prow[seg] != DT_PLAN_COMPUTE) continue;
           const int nt = key_set(G, qt, seg).ntiles();
           if (nt == 0) continue;
@@ -276,7 +337,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
                      idesc_qk, 1u);
             }
             mma_commit(&bars[C::bSFull + (g & 1)]);
-            if (pv_valid && !issue_pv()) { ok = false; break; }
+            DT_TR(0, g);
+            if (pv_valid && !issue_pv<DP>(bars, tmem, aV, pv_g, pv_seg, pv_first, pv_last, pv_precise, abort_flag,
+                                          p.status, lim)) {
+              ok = false;
+              break;
+            }
             pv_valid = 1; pv_g = g; pv_first = (i == 0); pv_last = (i == nt - 1); pv_seg = cseg;
             pv_precise = (G.window > 0 && seg == 0);
           }
@@ -284,14 +350,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         }
         mma_commit(&bars[C::bQEmpty]);
       }
-      if (ok && pv_valid) issue_pv();
+      if (ok && pv_valid)
+        issue_pv<DP>(bars, tmem, aV, pv_g, pv_seg, pv_first, pv_last, pv_precise, abort_flag, p.status, lim);
       // all MMAs of this CTA complete before tensor memory is freed
       mma_commit(&bars[C::bDrain]);
       volatile int never = 0;
       mbar_wait(&bars[C::bDrain], 0, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
     }
     __syncwarp();
+   }
   } else if (warp < 4) {
+    regs_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
     const int r = warp * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
@@ -304,7 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const QTile t = query_tile(G, qt);
       const int qrow = t.q0 + r;
       const int q1 = t.q0 + t.rows - 1;
-      for (int seg = 0; seg < G.P; ++seg) {
+      for (int j = 0; j < G.P; ++j) {
+        const int seg = visit_seg(G, idx, j);
         if (prow[seg] != DT_PLAN_COMPUTE) continue;
         const KeySet ks = key_set(G, qt, seg);
         const int nt = ks.ntiles();
@@ -313,9 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const bool precise = G.window > 0 && seg == 0;
         for (int i = 0; i < nt; ++i, ++g) {
           const uint32_t sb = g & 1;
+          if (warp == 0) DT_TR(1, g);
           if (!warp_wait(&bars[C::bSFull + sb], (g >> 1) & 1, abort_flag, p.status, lim)) goto sm_done;
+          if (warp == 0) DT_TR(2, g);
           tc_fence_after();
-          const int tile = ks.tile(i);
+          const int tile = visit_tile(ks, nt, idx, seg, i);
           const int k0 = ks.base + tile * kTile;
           const int kvalid = imin(kTile, ks.kend - k0);
           const uint32_t sc = tmem + lane_base + C::kColS + sb * 128;
@@ -329,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           if (G.window > 0)
             mask_kind = seg == 0 ? (wtile_inside(G, t.q0, q1, tile) ? 0 : 1)
                                  : (wtile_touches(G, t.q0, q1, tile) ? 2 : 0);
-          if (kvalid < kTile || mask_kind) {
+          const bool masked = kvalid < kTile || mask_kind != 0;
+          if (masked) {
 #pragma unroll
             for (int c = 0; c < 128; ++c) {
               const int key = k0 + c;
@@ -340,9 +413,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               if (!keep) sr[c] = f2u(kNegInf);
             }
           }
-          float mx = u2f(sr[0]);
+          // row max as 8 independent chains (a single 128-long chain is latency-bound)
+          float mx8[8];
 #pragma unroll
-          for (int c = 1; c < 128; ++c) mx = fmaxf(mx, u2f(sr[c]));
+          for (int j = 0; j < 8; ++j) mx8[j] = u2f(sr[j]);
+#pragma unroll
+          for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], u2f(sr[c]));
+          if (warp == 0) DT_TR(3, g);
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
           const float mx2 = mx * sl2;
           const float m_new = (i == 0) ? mx2 : ((mx2 > m_run + kRescaleThreshold) ? mx2 : m_run);
           const bool resc = (i > 0) && (m_new != m_run);
@@ -366,28 +445,61 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           }
           m_run = m_new;
           const float m_ref = (m_run == kNegInf) ? 0.f : m_run;
-          float lsum = 0.f;
+          float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent partial sums
+          if (!precise && !masked) {
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {        // 32 keys -> 16 packed bf16 pairs per chunk
-            uint32_t hi[16], lo[16];
+            for (int ch = 0; ch < 4; ++ch) {      // 32 keys -> 16 packed bf16 pairs per chunk
+              uint32_t hi[16];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int j = ch * 32 + 2 * c;
-              const float p0 = ex2(fmaf(u2f(sr[j]), sl2, -m_ref));
-              const float p1 = ex2(fmaf(u2f(sr[j + 1]), sl2, -m_ref));
-              lsum += p0 + p1;
-              hi[c] = pack_bf16x2(p0, p1);
-              // residual of the bf16 rounding, kept for the split-precision PV
-              lo[c] = pack_bf16x2(p0 - u2f(hi[c] << 16), p1 - u2f(hi[c] & 0xffff0000u));
+              for (int c = 0; c < 16; ++c) {
+                const int j = ch * 32 + 2 * c;
+                const float x0 = fmaf(u2f(sr[j]), sl2, -m_ref), x1 = fmaf(u2f(sr[j + 1]), sl2, -m_ref);
+                const bool emu = kEmuMod > 0 && (c % (kEmuMod > 0 ? kEmuMod : 1)) == kEmuMod - 1;
+                const float p0 = emu ? dt_exp2_fma(x0) : ex2(x0);
+                const float p1 = emu ? dt_exp2_fma(x1) : ex2(x1);
+                ls8[c & 7] += p0 + p1;
+                hi[c] = pack_bf16x2(p0, p1);
+              }
+              tmem_st16(sc + ch * 16, hi);
             }
-            tmem_st16(sc + ch * 16, hi);
-            if (precise) tmem_st16(sc + 64 + ch * 16, lo);
+          } else if (!precise) {                  // masked tile: -inf logits -> exactly 0 via MUFU
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t hi[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                const int j = ch * 32 + 2 * c;
+                const float p0 = ex2(fmaf(u2f(sr[j]), sl2, -m_ref));
+                const float p1 = ex2(fmaf(u2f(sr[j + 1]), sl2, -m_ref));
+                ls8[c & 7] += p0 + p1;
+                hi[c] = pack_bf16x2(p0, p1);
+              }
+              tmem_st16(sc + ch * 16, hi);
+            }
+          } else {
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t hi[16], lo[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                const int j = ch * 32 + 2 * c;
+                const float p0 = ex2(fmaf(u2f(sr[j]), sl2, -m_ref));
+                const float p1 = ex2(fmaf(u2f(sr[j + 1]), sl2, -m_ref));
+                ls8[c & 7] += p0 + p1;
+                hi[c] = pack_bf16x2(p0, p1);
+                // residual of the bf16 rounding, for the split-precision PV
+                lo[c] = pack_bf16x2(p0 - u2f(hi[c] << 16), p1 - u2f(hi[c] & 0xffff0000u));
+              }
+              tmem_st16(sc + ch * 16, hi);
+              tmem_st16(sc + 64 + ch * 16, lo);
+            }
           }
-          l_run += lsum;
+          l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars[C::bPFull + sb]);
+          if (warp == 0) DT_TR(4, g);
         }
         {
           const uint32_t st = cseg & 1;
@@ -403,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     }
   sm_done:;
   } else {
+    regs_inc<kRegsEpilogue>();
     // ------------------------------------------------------------ epilogue
     const int q4 = warp - 4;
     const int r = q4 * 32 + lane;
@@ -420,124 +533,140 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const bool valid = r < t.rows;
       float m_tot = kNegInf, l_tot = 0.f;
       bool have = false, use_r = false;
-      for (int seg = 0; seg < G.P; ++seg) {
-        const KeySet ks = key_set(G, qt, seg);
-        const int nt = ks.ntiles();
-        const size_t slot = (((size_t)seg * G.H + h) * G.S + qrow);
-        if (prow[seg] == DT_PLAN_COMPUTE) {
-          if (r == 0) { n_comp += counted_blocks(G, qt, seg); ++n_fresh; }
-          if (nt == 0) {           // empty key set: the identity state
-            if (G.window == 0 && valid) {
-              float4* dst = reinterpret_cast<float4*>(p.cache_O + slot * D);
-              for (int d = 0; d < D / 4; ++d) dst[d] = make_float4(0.f, 0.f, 0.f, 0.f);
-              p.cache_L[slot] = kNegInf;
-            }
-            continue;
-          }
-          const uint32_t st = cseg & 1;
-          if (!warp_wait(&bars[C::bStFull + st], (cseg >> 1) & 1, abort_flag, p.status, lim)) goto ep_done;
-          const float m_s = stat_m[st * 128 + r], l_s = stat_l[st * 128 + r];
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[C::bStFree + st]);
-          if (!warp_wait(&bars[C::bODSeg], cseg & 1, abort_flag, p.status, lim)) goto ep_done;
-          tc_fence_after();
-          const bool nonempty = l_s > 0.f;
-          const float inv_l = nonempty ? 1.f / l_s : 0.f;
-          float a, b, m_new;
-          if (!have) { m_new = m_s; a = 0.f; b = nonempty ? 1.f : 0.f; }
-          else {
-            m_new = nonempty ? fmaxf(m_tot, m_s) : m_tot;
-            a = ex2(m_tot - m_new);
-            b = nonempty ? ex2(m_s - m_new) : 0.f;
-          }
-          const float l_new = (have ? a * l_tot : 0.f) + b * l_s;
-          const bool make_r = G.window > 0 && seg == 1;
-          const float inv_tot = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
-          const float inv_new = l_new > 0.f ? 1.f / l_new : 0.f;
-#pragma unroll 1
-          for (int c0 = 0; c0 < DP; c0 += 16) {
-            uint32_t op[16], ot[16];
-            tmem_ld16(opart + c0, op);
-            tmem_ld16(otot + c0, ot);
-            tmem_wait_ld();
-            float nw[16];
+      // (1) cached states of the REUSE pairs: merged first, while the MMA and
+      //     softmax warps compute the item's first fresh state
+      for (int j = 0; j < G.P; ++j) {
+        const int seg = visit_seg(G, idx, j);
+        if (prow[seg] == DT_PLAN_COMPUTE) continue;
+        if (r == 0) { n_skip += counted_blocks(G, qt, seg); ++n_read; }
+        if (G.window > 0) { use_r = true; continue; }     // complement reused: add R at the end
+        const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
+        const float lse_c = valid ? p.cache_L[slot] : kNegInf;
+        const bool nonempty = lse_c > kNegInf;
+        float4 cv[DP / 4];                                  // the whole cached row, loads in flight together
+        const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float x = u2f(op[j]);
-              nw[j] = have ? fmaf(a, u2f(ot[j]), b * x) : b * x;
-            }
-            if (valid) {
-              if (G.window == 0) {
-                float* dst = p.cache_O + slot * D + c0;
+        for (int c = 0; c < DP / 4; ++c) cv[c] = (valid && 4 * c < D) ? src[c] : z4;
 #pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                  if (c0 + j < D)
-                    *reinterpret_cast<float4*>(dst + j) =
-                        make_float4(u2f(op[j]) * inv_l, u2f(op[j + 1]) * inv_l, u2f(op[j + 2]) * inv_l,
-                                    u2f(op[j + 3]) * inv_l);
-              } else if (make_r) {
-                float* dst = p.R + ((size_t)h * G.S + qrow) * D + c0;
-#pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                  if (c0 + j < D) {
-                    float4 v;
-                    v.x = nw[j] * inv_new - (have ? u2f(ot[j]) * inv_tot : 0.f);
-                    v.y = nw[j + 1] * inv_new - (have ? u2f(ot[j + 1]) * inv_tot : 0.f);
-                    v.z = nw[j + 2] * inv_new - (have ? u2f(ot[j + 2]) * inv_tot : 0.f);
-                    v.w = nw[j + 3] * inv_new - (have ? u2f(ot[j + 3]) * inv_tot : 0.f);
-                    *reinterpret_cast<float4*>(dst + j) = v;
-                  }
-              }
-            }
-            uint32_t o16[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) o16[j] = f2u(nw[j]);
-            tmem_st16(otot + c0, o16);
-          }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[C::bOFree]);
-          if (G.window == 0 && valid) p.cache_L[slot] = nonempty ? (m_s + lg2(l_s)) * kLn2 : kNegInf;
-          if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
-          have = have || nonempty;
-          ++cseg;
-        } else {
-          if (r == 0) { n_skip += counted_blocks(G, qt, seg); ++n_read; }
-          if (G.window > 0) { use_r = true; continue; }
-          const float lse_c = valid ? p.cache_L[slot] : kNegInf;
-          const bool nonempty = lse_c > kNegInf;
-          const float m_c = lse_c * kLog2e;
-          float a, b, m_new;
-          if (!have) { m_new = m_c; a = 0.f; b = nonempty ? 1.f : 0.f; }
-          else {
-            m_new = nonempty ? fmaxf(m_tot, m_c) : m_tot;
-            a = ex2(m_tot - m_new);
-            b = nonempty ? ex2(m_c - m_new) : 0.f;
-          }
-          const float l_new = (have ? a * l_tot : 0.f) + b;
-          const float* src = p.cache_O + slot * D;
-#pragma unroll 1
-          for (int c0 = 0; c0 < DP; c0 += 16) {
-            uint32_t ot[16];
-            tmem_ld16(otot + c0, ot);
-            float x[16];
-#pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-              float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (valid && nonempty && c0 + j < D) v = *reinterpret_cast<const float4*>(src + c0 + j);
-              x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
-            }
-            tmem_wait_ld();
-            uint32_t o16[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) o16[j] = f2u(have ? fmaf(a, u2f(ot[j]), b * x[j]) : b * x[j]);
-            tmem_st16(otot + c0, o16);
-          }
-          tmem_wait_st();
-          if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
-          have = have || nonempty;
+        for (int c = 0; c < DP / 4; ++c) cv[c] = nonempty ? cv[c] : z4;
+        const float m_c = lse_c * kLog2e;
+        float a, b, m_new;
+        if (!have) { m_new = m_c; a = 0.f; b = nonempty ? 1.f : 0.f; }
+        else {
+          m_new = nonempty ? fmaxf(m_tot, m_c) : m_tot;
+          a = ex2(m_tot - m_new);
+          b = nonempty ? ex2(m_c - m_new) : 0.f;
         }
+        const float l_new = (have ? a * l_tot : 0.f) + b;
+#pragma unroll
+        for (int c0 = 0; c0 < DP; c0 += 16) {
+          uint32_t ot[16], o16[16];
+          tmem_ld16(otot + c0, ot);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 16; jj += 4) {
+            const float4 x = cv[(c0 + jj) / 4];
+            o16[jj + 0] = f2u(have ? fmaf(a, u2f(ot[jj + 0]), b * x.x) : b * x.x);
+            o16[jj + 1] = f2u(have ? fmaf(a, u2f(ot[jj + 1]), b * x.y) : b * x.y);
+            o16[jj + 2] = f2u(have ? fmaf(a, u2f(ot[jj + 2]), b * x.z) : b * x.z);
+            o16[jj + 3] = f2u(have ? fmaf(a, u2f(ot[jj + 3]), b * x.w) : b * x.w);
+          }
+          tmem_st16(otot + c0, o16);
+        }
+        tmem_wait_st();
+        if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
+        have = have || nonempty;
+      }
+      // (2) fresh states, in the order the MMA produces them
+      for (int j = 0; j < G.P; ++j) {
+        const int seg = visit_seg(G, idx, j);
+        if (prow[seg] != DT_PLAN_COMPUTE) continue;
+        const int nt = key_set(G, qt, seg).ntiles();
+        const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
+        if (r == 0) { n_comp += counted_blocks(G, qt, seg); ++n_fresh; }
+        if (nt == 0) {             // empty key set: the identity state
+          if (G.window == 0 && valid) {
+            float4* dst = reinterpret_cast<float4*>(p.cache_O + slot * D);
+            for (int d = 0; d < D / 4; ++d) dst[d] = make_float4(0.f, 0.f, 0.f, 0.f);
+            p.cache_L[slot] = kNegInf;
+          }
+          continue;
+        }
+        const uint32_t st = cseg & 1;
+        if (!warp_wait(&bars[C::bStFull + st], (cseg >> 1) & 1, abort_flag, p.status, lim)) goto ep_done;
+        const float m_s = stat_m[st * 128 + r], l_s = stat_l[st * 128 + r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[C::bStFree + st]);
+        if (!warp_wait(&bars[C::bODSeg], cseg & 1, abort_flag, p.status, lim)) goto ep_done;
+        if (warp == 4) DT_TR(6, cseg);
+        tc_fence_after();
+        // O_part -> registers, then hand O_part straight back to the MMA warp
+        uint32_t op[DP];
+#pragma unroll
+        for (int c0 = 0; c0 < DP; c0 += 16) tmem_ld16p(opart + c0, op + c0);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[C::bOFree]);
+        if (warp == 4) DT_TR(7, cseg);
+        const bool nonempty = l_s > 0.f;
+        const float inv_l = nonempty ? 1.f / l_s : 0.f;
+        float a, b, m_new;
+        if (!have) { m_new = m_s; a = 0.f; b = nonempty ? 1.f : 0.f; }
+        else {
+          m_new = nonempty ? fmaxf(m_tot, m_s) : m_tot;
+          a = ex2(m_tot - m_new);
+          b = nonempty ? ex2(m_s - m_new) : 0.f;
+        }
+        const float l_new = (have ? a * l_tot : 0.f) + b * l_s;
+        const bool make_r = G.window > 0 && seg == 1;
+        const float inv_tot = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
+        const float inv_new = l_new > 0.f ? 1.f / l_new : 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < DP; c0 += 16) {
+          uint32_t ot[16];
+          tmem_ld16(otot + c0, ot);
+          tmem_wait_ld();
+          float nw[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const float x = u2f(op[c0 + jj]);
+            nw[jj] = have ? fmaf(a, u2f(ot[jj]), b * x) : b * x;
+          }
+          if (valid) {
+            if (G.window == 0) {
+              float* dst = p.cache_O + slot * D + c0;
+#pragma unroll
+              for (int jj = 0; jj < 16; jj += 4)
+                if (c0 + jj < D)
+                  *reinterpret_cast<float4*>(dst + jj) =
+                      make_float4(u2f(op[c0 + jj]) * inv_l, u2f(op[c0 + jj + 1]) * inv_l,
+                                  u2f(op[c0 + jj + 2]) * inv_l, u2f(op[c0 + jj + 3]) * inv_l);
+            } else if (make_r) {
+              float* dst = p.R + ((size_t)h * G.S + qrow) * D + c0;
+#pragma unroll
+              for (int jj = 0; jj < 16; jj += 4)
+                if (c0 + jj < D) {
+                  float4 v;
+                  v.x = nw[jj] * inv_new - (have ? u2f(ot[jj]) * inv_tot : 0.f);
+                  v.y = nw[jj + 1] * inv_new - (have ? u2f(ot[jj + 1]) * inv_tot : 0.f);
+                  v.z = nw[jj + 2] * inv_new - (have ? u2f(ot[jj + 2]) * inv_tot : 0.f);
+                  v.w = nw[jj + 3] * inv_new - (have ? u2f(ot[jj + 3]) * inv_tot : 0.f);
+                  *reinterpret_cast<float4*>(dst + jj) = v;
+                }
+            }
+          }
+          uint32_t o16[16];
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) o16[jj] = f2u(nw[jj]);
+          tmem_st16(otot + c0, o16);
+        }
+        tmem_wait_st();
+        if (G.window == 0 && valid) p.cache_L[slot] = nonempty ? (m_s + lg2(l_s)) * kLn2 : kNegInf;
+        if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
+        have = have || nonempty;
+        ++cseg;
       }
       // final: O = O_tot / l_tot (+ R), LSE = m_tot + log2(l_tot), in natural units
       {
@@ -602,6 +731,12 @@ int launch_dp(const AttnParams& kp, int grid, cudaStream_t stream) {
 }
 
 }  // namespace
+
+#ifdef DT_TRACE
+extern "C" __attribute__((visibility("default"))) int dt_debug_trace_set(uint64_t* d_buf) {
+  return cudaMemcpyToSymbol(g_dt_trace, &d_buf, sizeof(d_buf)) == cudaSuccess ? 0 : -4;
+}
+#endif
 
 int attn_fused_smem_bytes(int dp) {
   switch (dp) {
