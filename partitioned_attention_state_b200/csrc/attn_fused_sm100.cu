@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   const uint32_t tmem = *tmem_holder;
 
   if (warp >= 8) {
-   regs_dec<kRegsOther>();
+   regs_set<kLaunchRegs, kRegsOther>();
    if (warp == 9) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     __syncwarp();
    }
   } else if (warp < 4) {
-    regs_inc<kRegsSoftmax>();
+    regs_set<kLaunchRegs, kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
     const int r = warp * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
@@ -383,7 +383,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const bool precise = G.window > 0 && seg == 0;
         for (int i = 0; i < nt; ++i, ++g) {
           const uint32_t sb = g & 1;
-          if (warp == 0) DT_TR(1, g);
           if (!warp_wait(&bars[C::bSFull + sb], (g >> 1) & 1, abort_flag, p.status, lim)) goto sm_done;
           if (warp == 0) DT_TR(2, g);
           tc_fence_after();
@@ -397,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           tmem_ld32(sc + 64, sr + 64);
           tmem_ld32(sc + 96, sr + 96);
           tmem_wait_ld();
+          if (warp == 0) DT_TR(1, g);
           int mask_kind = 0;   // 1: keep |i-j| <= hw, 2: keep |i-j| > hw
           if (G.window > 0)
             mask_kind = seg == 0 ? (wtile_inside(G, t.q0, q1, tile) ? 0 : 1)
@@ -494,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               tmem_st16(sc + 64 + ch * 16, lo);
             }
           }
+          if (warp == 0) DT_TR(6, g);
           l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
           tmem_wait_st();
           tc_fence_before();
@@ -515,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     }
   sm_done:;
   } else {
-    regs_inc<kRegsEpilogue>();
+    regs_set<kLaunchRegs, kRegsEpilogue>();
     // ------------------------------------------------------------ epilogue
     const int q4 = warp - 4;
     const int r = q4 * 32 + lane;
@@ -599,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[C::bStFree + st]);
         if (!warp_wait(&bars[C::bODSeg], cseg & 1, abort_flag, p.status, lim)) goto ep_done;
-        if (warp == 4) DT_TR(6, cseg);
+
         tc_fence_after();
         // O_part -> registers, then hand O_part straight back to the MMA warp
         uint32_t op[DP];

@@ -47,6 +47,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe: has the phase of `parity` completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+#ifndef DT_WAIT_MODE
+#define DT_WAIT_MODE 0
+#endif
+// try_wait with a suspend-time hint (ns): the thread sleeps until the phase
+// completes or the hint elapses, instead of re-polling.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of `parity` to complete.  Returns false (and
 // leaves the caller to bail out) when *abort is raised by another role or the
 // wait exceeds limit_ns, in which case it raises *abort itself and records
@@ -56,9 +86,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
+#if DT_WAIT_MODE == 1
+    if (mbar_try_wait_hint(bar, parity, 200000u)) return true;
+#elif DT_WAIT_MODE == 2
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      if (mbar_try_wait(bar, parity)) return true;
+      __nanosleep(32);
+    }
+#else
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+#endif
     if (*abort) return false;
     if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
@@ -190,6 +230,14 @@ template <uint32_t N>
 __device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
 template <uint32_t N>
 __device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+// Move this warpgroup from the launch count `From` to `To` registers per
+// thread: .inc may only raise and .dec only lower the count.
+template <uint32_t From, uint32_t To>
+__device__ __forceinline__ void regs_set() {
+  static_assert(To % 8 == 0 && To >= 24 && To <= 256, "setmaxnreg range");
+  if constexpr (To > From) regs_inc<To>();
+  else if constexpr (To < From) regs_dec<To>();
+}
 
 // Shared-memory matrix descriptor (tcgen05 "matrix descriptor"): start
 // address, leading/stride byte offsets (>>4), fixed version bits 46-47 = 1,
