@@ -114,6 +114,7 @@ extern "C" int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_p
   kp.counters = d_counters;
   kp.status = d_status;
   kp.H = p->H; kp.S = p->S; kp.D = p->D; kp.P = win ? 1 : p->P; kp.window = win ? p->window : 0;
+  kp.geom = G;
   kp.n_items = p->H * G.nqt;
   kp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->D));
   kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();

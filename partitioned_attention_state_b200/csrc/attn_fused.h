@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "geometry.h"
+
 namespace dt {
 
 struct AttnParams {
@@ -19,6 +21,7 @@ struct AttnParams {
   int64_t* counters;
   int32_t* status;
   int H, S, D, P, window;           // P: partitions (ignored in window mode)
+  Geom geom;                        // make_geom(H, S, D, P, window), read from the parameter bank
   int n_items;                      // H * nqt
   float scale_log2;                 // log2(e) / sqrt(D)
   uint64_t wait_limit_ns;

@@ -17,19 +17,26 @@
 // persistent (one CTA per SM) and strides over items head-major so the CTAs
 // running together share a head's K/V in L2; each item visits its key sets and
 // key tiles in a rotated order so those CTAs do not read the same tile at the
-// same moment.  Per CTA, 12 warps (3 warpgroups, registers rebalanced with
+// same moment.  Per CTA, 16 warps (4 warpgroups, registers rebalanced with
 // setmaxnreg):
-//   warps 0-3  softmax:   S (TMEM) -> P (bf16, written back over S in TMEM),
-//                         running row max/sum, conditional O rescale
-//   warps 4-7  epilogue:  per reused key set (first, off the critical path):
+//   warps 0-7   softmax:  two warps per SM sub-partition, each owning 16 rows
+//                         of the tile (16-lane TMEM accesses; a thread holds 2
+//                         rows x 32 columns).  S (TMEM) -> P (bf16, written back
+//                         over S in TMEM), running row max/sum, conditional O
+//                         rescale.  Two warps per sub-partition keep the
+//                         exponential unit busy while the other warp loads S,
+//                         reduces its max or stores P.
+//   warps 8-11  epilogue: per reused key set (first, off the critical path):
 //                         cached state composed into O_tot (TMEM); per computed
 //                         key set: O_part (TMEM) -> registers (O_part released at
 //                         once) -> normalised fresh state -> cache slot, composed
 //                         into O_tot; per item: O_tot -> O (bf16), LSE
-//   warp 8     MMA:       tcgen05.mma S = Q K^T (smem x smem), O_part += P V
+//   warp 12     MMA:      tcgen05.mma S = Q K^T (smem x smem), O_part += P V
 //                         (P from TMEM, V from smem); TMEM alloc/free
-//   warp 9     TMA:       Q once per item, K/V tiles into an NS-stage ring
-//   warps 10-11 idle (complete the third warpgroup)
+//   warp 13     TMA:      Q once per item, K tiles into an NS-stage ring
+//   warp 14     TMA:      V tiles into an NS-stage ring (released separately
+//                         from K: a K stage frees as soon as its QK^T is done)
+//   warp 15     idle (completes the fourth warpgroup)
 // Tensor memory (512 columns): S/P double buffer [0,256), O_part [256,256+DP),
 // O_tot [256+DP, 256+2*DP).  DP = head dim padded to a multiple of 16 (72 -> 80):
 // a 64-column block uses the 128-byte swizzle, the 16-column tail of D=72 the
@@ -59,15 +66,15 @@ namespace {
 
 using namespace sm100;
 
-// 3 warpgroups: softmax (warps 0-3), epilogue (4-7), MMA (8) + TMA (9) + 2 idle.
-constexpr int kThreads = 384;
-// Registers per thread at launch (ptxas: 65536 / 384, rounded down to 8; the
-// build checks it) and the per-warpgroup split after setmaxnreg.  The split
-// must fit the launch pool: 128 * (kRegsSoftmax + kRegsEpilogue + kRegsOther)
-// <= kThreads * kLaunchRegs.
-constexpr int kLaunchRegs = 168;
-constexpr int kRegsSoftmax = 208, kRegsEpilogue = 224, kRegsOther = 64;
-static_assert(128 * (kRegsSoftmax + kRegsEpilogue + kRegsOther) <= kThreads * kLaunchRegs, "register split");
+// 4 warpgroups: softmax (warps 0-7), epilogue (8-11), MMA (12) + TMA (13, 14) + idle (15).
+constexpr int kThreads = 512;
+constexpr int kWarpEpi = 8, kWarpMma = 12, kWarpTmaK = 13, kWarpTmaV = 14;
+// Registers per thread at launch (ptxas: 65536 / 512; the build checks it) and
+// the per-warpgroup split after setmaxnreg.  The split must fit the launch
+// pool: 128 * (2 * kRegsSoftmax + kRegsEpilogue + kRegsOther) <= kThreads * kLaunchRegs.
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsSoftmax = 128, kRegsEpilogue = 192, kRegsOther = 64;
+static_assert(128 * (2 * kRegsSoftmax + kRegsEpilogue + kRegsOther) <= kThreads * kLaunchRegs, "register split");
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // drains use a fixed limit
 __device__ __forceinline__ float neg_inf() { return -__int_as_float(0x7f800000); }
 #define kNegInf (neg_inf())
@@ -102,25 +109,17 @@ struct Cfg {
   static constexpr int kColOtot = 256 + DP;
   static_assert(kColOtot + DP <= 512, "tensor memory budget");
   // barrier indices
-  static constexpr int bQFull = 0, bQEmpty = 1, bKFull = 2, bVFull = 2 + kStages, bKVEmpty = 2 + 2 * kStages,
-                       bSFull = 2 + 3 * kStages, bPFull = bSFull + 2, bODone = bPFull + 2, bODSeg = bODone + 1,
-                       bOFree = bODSeg + 1, bStFull = bOFree + 1, bStFree = bStFull + 2, bDrain = bStFree + 2,
-                       kNumBars = bDrain + 1;
+  static constexpr int bQFull = 0, bQEmpty = 1, bKFull = 2, bVFull = 2 + kStages, bKEmpty = 2 + 2 * kStages,
+                       bVEmpty = 2 + 3 * kStages, bSFull = 2 + 4 * kStages, bPFull = bSFull + 2,
+                       bODone = bPFull + 2, bODSeg = bODone + 1, bOFree = bODSeg + 1, bStFull = bOFree + 1,
+                       bStFree = bStFull + 2, bDrain = bStFree + 2, kNumBars = bDrain + 1;
   static constexpr int kStatsBytes = 2 * 2 * 128 * 4;
   static constexpr int kSmem = kTileBytes * (1 + 2 * kStages) + kStatsBytes + kNumBars * 8 + 16;
 };
 
-// Exponentials of an unmasked tile: when kEmuMod > 0 every kEmuMod-th pair is
-// evaluated on the FMA pipe instead of MUFU.  Off: with one or two softmax
-// warps per SM sub-partition the loop is latency-bound, not MUFU-bound, and
-// the polynomial only lengthens it (measured).
+// Exponentials of an unmasked tile: when kEmuMod > 0 every kEmuMod-th
+// repetition (4 values) is evaluated on the FMA pipe instead of MUFU.
 constexpr int kEmuMod = 0;
-
-// Two non-negative finite floats -> packed bf16x2 (lo = a), rounded half up,
-// with integer ops (keeps the conversion off the MUFU/XU pipe).
-__device__ __forceinline__ uint32_t pack_bf16x2_rhu(float a, float b) {
-  return __byte_perm(__float_as_uint(a) + 0x8000u, __float_as_uint(b) + 0x8000u, 0x7632);
-}
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
@@ -135,9 +134,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return ok != 0;
 }
 
+template <bool WIN>
 __device__ __forceinline__ bool item_has_compute(const Geom& G, int qt, const uint8_t* prow) {
   for (int s = 0; s < G.P; ++s)
-    if (prow[s] == DT_PLAN_COMPUTE && key_set(G, qt, s).ntiles() > 0) return true;
+    if (prow[s] == DT_PLAN_COMPUTE && key_set<WIN>(G, qt, s).ntiles() > 0) return true;
   return false;
 }
 
@@ -145,8 +145,9 @@ __device__ __forceinline__ bool item_has_compute(const Geom& G, int qt, const ui
 // compose associatively and commutatively and the online softmax is order
 // free, so any order gives the same result; rotating the start per item keeps
 // the CTAs that run together from streaming the same K/V tile at once.
+template <bool WIN>
 __device__ __forceinline__ int visit_seg(const Geom& G, int idx, int j) {
-  if (G.window > 0) return j;                 // window set before its complement
+  if (WIN) return j;                 // window set before its complement
   int s = j + idx % G.P;
   return s >= G.P ? s - G.P : s;
 }
@@ -185,13 +186,13 @@ __device__ __forceinline__ bool issue_pv(uint64_t* bars, uint32_t tmem, uint32_t
       if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + 64 + kk * 8, vdt, idesc_pvt, 1u);
     }
   }
-  mma_commit(&bars[C::bKVEmpty + st]);
+  mma_commit(&bars[C::bVEmpty + st]);
   mma_commit(&bars[C::bODone]);
   if (last) mma_commit(&bars[C::bODSeg]);
   return true;
 }
 
-template <int DP>
+template <int DP, bool WIN>
 __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<DP>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -209,23 +210,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const Geom G = make_geom(p.H, p.S, p.D, p.P, p.window);
+  const Geom& G = p.geom;
   const uint64_t lim = p.wait_limit_ns;
 
-  if (warp == 9 && lane == 0) {
+  if (warp == kWarpTmaK && lane == 0) {
     for (int i = 0; i < C::kNumBars; ++i) mbar_init(&bars[i], 1);
-    mbar_init(&bars[C::bPFull + 0], 4);
-    mbar_init(&bars[C::bPFull + 1], 4);
-    mbar_init(&bars[C::bOFree], 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[C::bStFull + i], 4);
-      mbar_init(&bars[C::bStFree + i], 4);
+      mbar_init(&bars[C::bPFull + i], 8);     // one arrival per softmax warp
+      mbar_init(&bars[C::bStFull + i], 8);
+      mbar_init(&bars[C::bStFree + i], 4);    // one arrival per epilogue warp
     }
+    mbar_init(&bars[C::bOFree], 4);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async();
   }
-  if (warp == 8) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
@@ -234,65 +234,75 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp >= 8) {
+  if (warp >= kWarpMma) {
    regs_set<kLaunchRegs, kRegsOther>();
-   if (warp == 9) {
-    // ------------------------------------------------------------ TMA producer
+   if (warp == kWarpTmaK || warp == kWarpTmaV) {
+    // ------------------------------------------------------------ TMA producers
+    // Warp 13 loads Q (once per item) and the K ring, warp 14 the V ring; both
+    // walk the same tile sequence.
     if (lane == 0) {
-      prefetch_tmap(&p.tmQ); prefetch_tmap(&p.tmK); prefetch_tmap(&p.tmV);
-      if (C::kTail) { prefetch_tmap(&p.tmQt); prefetch_tmap(&p.tmKt); prefetch_tmap(&p.tmVt); }
+      const bool is_k = warp == kWarpTmaK;
+      const CUtensorMap* tm = is_k ? &p.tmK : &p.tmV;
+      const CUtensorMap* tmt = is_k ? &p.tmKt : &p.tmVt;
+      uint8_t* ring = is_k ? sK : sV;
+      uint64_t* full = &bars[is_k ? C::bKFull : C::bVFull];
+      uint64_t* empty = &bars[is_k ? C::bKEmpty : C::bVEmpty];
+      prefetch_tmap(tm);
+      if (C::kTail) prefetch_tmap(tmt);
+      if (is_k) { prefetch_tmap(&p.tmQ); if (C::kTail) prefetch_tmap(&p.tmQt); }
+      // K/V tiles are re-read by every query tile of the head: keep them in L2
+      // against the streaming state-cache traffic; a Q tile is read once.
+      const uint64_t pol_keep = l2_policy_evict_last(), pol_once = l2_policy_evict_first();
       uint32_t g = 0, nq = 0;
       for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
         const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
         const uint8_t* prow = p.plan + (size_t)qt * G.P;
-        if (!item_has_compute(G, qt, prow)) continue;
-        const QTile t = query_tile(G, qt);
-        if (nq > 0 && !mbar_wait(&bars[C::bQEmpty], (nq - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
-          goto tma_done;
-        mbar_arrive_expect_tx(&bars[C::bQFull], C::kTileBytes);
-        for (int c = 0; c < C::kN64; ++c) tma_load_3d(sQ + c * C::kBlk, &p.tmQ, &bars[C::bQFull], 64 * c, t.q0, h);
-        if (C::kTail) tma_load_3d(sQ + C::kN64 * C::kBlk, &p.tmQt, &bars[C::bQFull], 64 * C::kN64, t.q0, h);
-        ++nq;
+        if (!item_has_compute<WIN>(G, qt, prow)) continue;
+        if (is_k) {
+          const QTile t = query_tile<WIN>(G, qt);
+          if (nq > 0 && !mbar_wait(&bars[C::bQEmpty], (nq - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
+            goto tma_done;
+          mbar_arrive_expect_tx(&bars[C::bQFull], C::kTileBytes);
+          for (int c = 0; c < C::kN64; ++c)
+            tma_load_3d_hint(sQ + c * C::kBlk, &p.tmQ, &bars[C::bQFull], 64 * c, t.q0, h, pol_once);
+          if (C::kTail)
+            tma_load_3d_hint(sQ + C::kN64 * C::kBlk, &p.tmQt, &bars[C::bQFull], 64 * C::kN64, t.q0, h, pol_once);
+          ++nq;
+        }
         for (int j = 0; j < G.P; ++j) {
-          const int seg = visit_seg(G, idx, j);
+          const int seg = visit_seg<WIN>(G, idx, j);
           if (prow[seg] != DT_PLAN_COMPUTE) continue;
-          const KeySet ks = key_set(G, qt, seg);
+          const KeySet ks = key_set<WIN>(G, qt, seg);
           const int nt = ks.ntiles();
           for (int i = 0; i < nt; ++i, ++g) {
             const int st = g % C::kStages;
             if (g >= (uint32_t)C::kStages &&
-                !mbar_wait(&bars[C::bKVEmpty + st], ((g / C::kStages) - 1) & 1, abort_flag, p.status,
-                           DT_ERR_TIMEOUT, lim))
+                !mbar_wait(&empty[st], ((g / C::kStages) - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
               goto tma_done;
             const int row0 = ks.base + visit_tile(ks, nt, idx, seg, i) * kTile;
-            uint8_t* dk = sK + st * C::kTileBytes;
-            uint8_t* dv = sV + st * C::kTileBytes;
-            mbar_arrive_expect_tx(&bars[C::bKFull + st], C::kTileBytes);
-            for (int c = 0; c < C::kN64; ++c) tma_load_3d(dk + c * C::kBlk, &p.tmK, &bars[C::bKFull + st], 64 * c, row0, h);
-            if (C::kTail) tma_load_3d(dk + C::kN64 * C::kBlk, &p.tmKt, &bars[C::bKFull + st], 64 * C::kN64, row0, h);
-            mbar_arrive_expect_tx(&bars[C::bVFull + st], C::kTileBytes);
-            for (int c = 0; c < C::kN64; ++c) tma_load_3d(dv + c * C::kBlk, &p.tmV, &bars[C::bVFull + st], 64 * c, row0, h);
-            if (C::kTail) tma_load_3d(dv + C::kN64 * C::kBlk, &p.tmVt, &bars[C::bVFull + st], 64 * C::kN64, row0, h);
+            uint8_t* dst = ring + st * C::kTileBytes;
+            DT_TR(is_k ? 8 : 9, g);
+            mbar_arrive_expect_tx(&full[st], C::kTileBytes);
+            for (int c = 0; c < C::kN64; ++c) tma_load_3d_hint(dst + c * C::kBlk, tm, &full[st], 64 * c, row0, h, pol_keep);
+            if (C::kTail) tma_load_3d_hint(dst + C::kN64 * C::kBlk, tmt, &full[st], 64 * C::kN64, row0, h, pol_keep);
           }
         }
       }
     tma_done:
-      // let every copy this CTA started land before its shared memory goes away
+      // let every copy this warp started land before shared memory goes away
       for (int s = 0; s < C::kStages; ++s) {
         if ((uint32_t)s < g) {
           const uint32_t last = g - 1 - ((g - 1 - s) % C::kStages);   // latest tile that used stage s
-          const uint32_t ph = (last / C::kStages) & 1;
           volatile int never = 0;
-          mbar_wait(&bars[C::bKFull + s], ph, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
-          mbar_wait(&bars[C::bVFull + s], ph, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
+          mbar_wait(&full[s], (last / C::kStages) & 1, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
         }
       }
-      if (nq > 0) {
+      if (is_k && nq > 0) {
         volatile int never = 0;
         mbar_wait(&bars[C::bQFull], (nq - 1) & 1, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
       }
     }
-   } else if (warp == 8) {
+   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
@@ -307,17 +317,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint8_t* prow = p.plan + (size_t)qt * G.P;
-        if (!item_has_compute(G, qt, prow)) continue;
+        if (!item_has_compute<WIN>(G, qt, prow)) continue;
         if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
         ++nq;
         tc_fence_after();
         for (int j = 0; j < G.P && ok; ++j) {
-          const int seg = visit_seg(G, idx, j);
+          const int seg = visit_seg<WIN>(G, idx, j);
           if (prow[seg] != DT_PLAN_COMPUTE) continue;
-          const int nt = key_set(G, qt, seg).ntiles();
+          const int nt = key_set<WIN>(G, qt, seg).ntiles();
           if (nt == 0) continue;
           for (int i = 0; i < nt; ++i, ++g) {
             const int st = g % C::kStages;
+            DT_TR(10, g);
             if (!mbar_wait(&bars[C::bKFull + st], (g / C::kStages) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) {
               ok = false;
               break;
@@ -337,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
                      idesc_qk, 1u);
             }
             mma_commit(&bars[C::bSFull + (g & 1)]);
+            mma_commit(&bars[C::bKEmpty + st]);
             DT_TR(0, g);
             if (pv_valid && !issue_pv<DP>(bars, tmem, aV, pv_g, pv_seg, pv_first, pv_last, pv_precise, abort_flag,
                                           p.status, lim)) {
@@ -344,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               break;
             }
             pv_valid = 1; pv_g = g; pv_first = (i == 0); pv_last = (i == nt - 1); pv_seg = cseg;
-            pv_precise = (G.window > 0 && seg == 0);
+            pv_precise = (WIN && seg == 0);
           }
           ++cseg;
         }
@@ -359,28 +371,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     }
     __syncwarp();
    }
-  } else if (warp < 4) {
+  } else if (warp < kWarpEpi) {
     regs_set<kLaunchRegs, kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // Warp w owns tile rows rbase .. rbase+15 (TMEM lanes of its sub-partition
+    // w % 4); thread t holds rows ra = rbase + t/4 and rb = ra + 8 at columns
+    // 8i + 2(t%4) + {0,1}, i = 0..15.  The P pair of those two columns is P
+    // column 4i + t%4, which the 16x128b store writes from the same thread.
+    const int rbase = (warp & 3) * 32 + (warp >> 2) * 16;
+    const int ra = rbase + (lane >> 2), rb = ra + 8;
+    const int cq = 2 * (lane & 3);
+    const uint32_t lane_base = static_cast<uint32_t>(rbase) << 16;
     const float sl2 = p.scale_log2;
     uint32_t g = 0, cseg = 0;
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const int qt = idx - (idx / G.nqt) * G.nqt;
       const uint8_t* prow = p.plan + (size_t)qt * G.P;
-      if (!item_has_compute(G, qt, prow)) continue;
-      const QTile t = query_tile(G, qt);
-      const int qrow = t.q0 + r;
+      if (!item_has_compute<WIN>(G, qt, prow)) continue;
+      const QTile t = query_tile<WIN>(G, qt);
+      const int qa = t.q0 + ra, qb = t.q0 + rb;
       const int q1 = t.q0 + t.rows - 1;
       for (int j = 0; j < G.P; ++j) {
-        const int seg = visit_seg(G, idx, j);
+        const int seg = visit_seg<WIN>(G, idx, j);
         if (prow[seg] != DT_PLAN_COMPUTE) continue;
-        const KeySet ks = key_set(G, qt, seg);
+        const KeySet ks = key_set<WIN>(G, qt, seg);
         const int nt = ks.ntiles();
         if (nt == 0) continue;
-        float m_run = kNegInf, l_run = 0.f;
-        const bool precise = G.window > 0 && seg == 0;
+        // running max (log2 units) and partial row sums of rows ra, rb
+        float ma = kNegInf, mb = kNegInf;
+        float la[4] = {0.f, 0.f, 0.f, 0.f}, lb[4] = {0.f, 0.f, 0.f, 0.f};
+        const bool precise = WIN && seg == 0;
         for (int i = 0; i < nt; ++i, ++g) {
           const uint32_t sb = g & 1;
           if (!warp_wait(&bars[C::bSFull + sb], (g >> 1) & 1, abort_flag, p.status, lim)) goto sm_done;
@@ -390,112 +410,103 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           const int k0 = ks.base + tile * kTile;
           const int kvalid = imin(kTile, ks.kend - k0);
           const uint32_t sc = tmem + lane_base + C::kColS + sb * 128;
-          uint32_t sr[128];
-          tmem_ld32(sc + 0, sr);
-          tmem_ld32(sc + 32, sr + 32);
-          tmem_ld32(sc + 64, sr + 64);
-          tmem_ld32(sc + 96, sr + 96);
+          uint32_t sr[64];
+          tmem_ld_16x256b_x8(sc, sr);
+          tmem_ld_16x256b_x8(sc + 64, sr + 32);
           tmem_wait_ld();
           if (warp == 0) DT_TR(1, g);
           int mask_kind = 0;   // 1: keep |i-j| <= hw, 2: keep |i-j| > hw
-          if (G.window > 0)
+          if (WIN)
             mask_kind = seg == 0 ? (wtile_inside(G, t.q0, q1, tile) ? 0 : 1)
                                  : (wtile_touches(G, t.q0, q1, tile) ? 2 : 0);
           const bool masked = kvalid < kTile || mask_kind != 0;
           if (masked) {
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
+            for (int e = 0; e < 64; ++e) {
+              const int c = 8 * (e >> 2) + cq + (e & 1);
               const int key = k0 + c;
-              const int dist = qrow > key ? qrow - key : key - qrow;
+              const int q = (e & 2) ? qb : qa;
+              const int dist = q > key ? q - key : key - q;
               bool keep = c < kvalid;
               if (mask_kind == 1) keep = keep && dist <= G.hw;
               if (mask_kind == 2) keep = keep && dist > G.hw;
-              if (!keep) sr[c] = f2u(kNegInf);
+              if (!keep) sr[e] = f2u(kNegInf);
             }
           }
-          // row max as 8 independent chains (a single 128-long chain is latency-bound)
-          float mx8[8];
+          // row maxima: two chains per row, then across the 4 threads of a row
+          float xa0 = fmaxf(u2f(sr[0]), u2f(sr[1])), xa1 = fmaxf(u2f(sr[4]), u2f(sr[5]));
+          float xb0 = fmaxf(u2f(sr[2]), u2f(sr[3])), xb1 = fmaxf(u2f(sr[6]), u2f(sr[7]));
 #pragma unroll
-          for (int j = 0; j < 8; ++j) mx8[j] = u2f(sr[j]);
-#pragma unroll
-          for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], u2f(sr[c]));
+          for (int r4 = 2; r4 < 16; r4 += 2) {
+            xa0 = max3f(xa0, u2f(sr[4 * r4]), u2f(sr[4 * r4 + 1]));
+            xa1 = max3f(xa1, u2f(sr[4 * r4 + 4]), u2f(sr[4 * r4 + 5]));
+            xb0 = max3f(xb0, u2f(sr[4 * r4 + 2]), u2f(sr[4 * r4 + 3]));
+            xb1 = max3f(xb1, u2f(sr[4 * r4 + 6]), u2f(sr[4 * r4 + 7]));
+          }
+          float mxa = fmaxf(xa0, xa1), mxb = fmaxf(xb0, xb1);
+          mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
+          mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
+          mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
+          mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
           if (warp == 0) DT_TR(3, g);
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-          const float mx2 = mx * sl2;
-          const float m_new = (i == 0) ? mx2 : ((mx2 > m_run + kRescaleThreshold) ? mx2 : m_run);
-          const bool resc = (i > 0) && (m_new != m_run);
-          if (__any_sync(0xffffffffu, resc)) {
+          const float mxa2 = mxa * sl2, mxb2 = mxb * sl2;
+          const float na = (i == 0) ? mxa2 : ((mxa2 > ma + kRescaleThreshold) ? mxa2 : ma);
+          const float nb = (i == 0) ? mxb2 : ((mxb2 > mb + kRescaleThreshold) ? mxb2 : mb);
+          const bool resa = (i > 0) && (na != ma), resb = (i > 0) && (nb != mb);
+          if (__any_sync(0xffffffffu, resa || resb)) {
             // O_part holds the previous tiles' sum: wait for its last PV, then rescale
             if (!warp_wait(&bars[C::bODone], (g - 1) & 1, abort_flag, p.status, lim)) goto sm_done;
             tc_fence_after();
-            const float alpha = resc ? ex2(m_run - m_new) : 1.f;
+            const float alpha_a = resa ? ex2(ma - na) : 1.f, alpha_b = resb ? ex2(mb - nb) : 1.f;
             const uint32_t oc = tmem + lane_base + C::kColOpart;
-#pragma unroll
+#pragma unroll 1
             for (int c0 = 0; c0 < DP; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld16(oc + c0, o);
+              uint32_t o[8];
+              tmem_ld_16x256b_x2(oc + c0, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 16; ++j) o[j] = f2u(u2f(o[j]) * alpha);
-              tmem_st16(oc + c0, o);
+              for (int e = 0; e < 8; ++e) o[e] = f2u(u2f(o[e]) * ((e & 2) ? alpha_b : alpha_a));
+              tmem_st_16x256b_x2(oc + c0, o);
             }
             tmem_wait_st();
-            l_run *= alpha;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) { la[k] *= alpha_a; lb[k] *= alpha_b; }
           }
-          m_run = m_new;
-          const float m_ref = (m_run == kNegInf) ? 0.f : m_run;
-          float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent partial sums
-          if (!precise && !masked) {
+          ma = na; mb = nb;
+          const float mra = (ma == kNegInf) ? 0.f : ma, mrb = (mb == kNegInf) ? 0.f : mb;
+          // exponentials, 8 repetitions (32 P columns) per TMEM store
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {      // 32 keys -> 16 packed bf16 pairs per chunk
-              uint32_t hi[16];
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t ph[16];
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const int j = ch * 32 + 2 * c;
-                const float x0 = fmaf(u2f(sr[j]), sl2, -m_ref), x1 = fmaf(u2f(sr[j + 1]), sl2, -m_ref);
-                const bool emu = kEmuMod > 0 && (c % (kEmuMod > 0 ? kEmuMod : 1)) == kEmuMod - 1;
-                const float p0 = emu ? dt_exp2_fma(x0) : ex2(x0);
-                const float p1 = emu ? dt_exp2_fma(x1) : ex2(x1);
-                ls8[c & 7] += p0 + p1;
-                hi[c] = pack_bf16x2(p0, p1);
+            for (int r4 = 0; r4 < 8; ++r4) {
+              const int e = 4 * (8 * hf + r4);
+              const float x0 = fmaf(u2f(sr[e]), sl2, -mra), x1 = fmaf(u2f(sr[e + 1]), sl2, -mra);
+              const float x2 = fmaf(u2f(sr[e + 2]), sl2, -mrb), x3 = fmaf(u2f(sr[e + 3]), sl2, -mrb);
+              const bool emu = kEmuMod > 0 && !masked && !precise && (r4 % (kEmuMod > 0 ? kEmuMod : 1)) == kEmuMod - 1;
+              const float p0 = emu ? dt_exp2_fma(x0) : ex2(x0), p1 = emu ? dt_exp2_fma(x1) : ex2(x1);
+              const float p2 = emu ? dt_exp2_fma(x2) : ex2(x2), p3 = emu ? dt_exp2_fma(x3) : ex2(x3);
+              la[r4 & 3] += p0 + p1;
+              lb[r4 & 3] += p2 + p3;
+              ph[2 * r4] = pack_bf16x2(p0, p1);
+              ph[2 * r4 + 1] = pack_bf16x2(p2, p3);
+              if (precise) {                      // bf16 residuals overwrite the consumed logits
+                sr[e] = pack_bf16x2(p0 - u2f(ph[2 * r4] << 16), p1 - u2f(ph[2 * r4] & 0xffff0000u));
+                sr[e + 1] = pack_bf16x2(p2 - u2f(ph[2 * r4 + 1] << 16), p3 - u2f(ph[2 * r4 + 1] & 0xffff0000u));
               }
-              tmem_st16(sc + ch * 16, hi);
             }
-          } else if (!precise) {                  // masked tile: -inf logits -> exactly 0 via MUFU
+            tmem_st_16x128b_x8(sc + 32 * hf, ph);
+            if (precise) {                        // P_lo in columns 64..127
+              uint32_t pl[16];
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-              uint32_t hi[16];
-#pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const int j = ch * 32 + 2 * c;
-                const float p0 = ex2(fmaf(u2f(sr[j]), sl2, -m_ref));
-                const float p1 = ex2(fmaf(u2f(sr[j + 1]), sl2, -m_ref));
-                ls8[c & 7] += p0 + p1;
-                hi[c] = pack_bf16x2(p0, p1);
+              for (int r4 = 0; r4 < 8; ++r4) {
+                pl[2 * r4] = sr[4 * (8 * hf + r4)];
+                pl[2 * r4 + 1] = sr[4 * (8 * hf + r4) + 1];
               }
-              tmem_st16(sc + ch * 16, hi);
-            }
-          } else {
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-              uint32_t hi[16], lo[16];
-#pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                const int j = ch * 32 + 2 * c;
-                const float p0 = ex2(fmaf(u2f(sr[j]), sl2, -m_ref));
-                const float p1 = ex2(fmaf(u2f(sr[j + 1]), sl2, -m_ref));
-                ls8[c & 7] += p0 + p1;
-                hi[c] = pack_bf16x2(p0, p1);
-                // residual of the bf16 rounding, for the split-precision PV
-                lo[c] = pack_bf16x2(p0 - u2f(hi[c] << 16), p1 - u2f(hi[c] & 0xffff0000u));
-              }
-              tmem_st16(sc + ch * 16, hi);
-              tmem_st16(sc + 64 + ch * 16, lo);
+              tmem_st_16x128b_x8(sc + 64 + 32 * hf, pl);
             }
           }
           if (warp == 0) DT_TR(6, g);
-          l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -503,11 +514,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           if (warp == 0) DT_TR(4, g);
         }
         {
+          float sa = ((la[0] + la[1]) + (la[2] + la[3])), sbm = ((lb[0] + lb[1]) + (lb[2] + lb[3]));
+          sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+          sbm += __shfl_xor_sync(0xffffffffu, sbm, 1);
+          sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+          sbm += __shfl_xor_sync(0xffffffffu, sbm, 2);
           const uint32_t st = cseg & 1;
           if (cseg >= 2 && !warp_wait(&bars[C::bStFree + st], ((cseg >> 1) - 1) & 1, abort_flag, p.status, lim))
             goto sm_done;
-          stat_m[st * 128 + r] = m_run;
-          stat_l[st * 128 + r] = l_run;
+          if ((lane & 3) == 0) {
+            stat_m[st * 128 + ra] = ma;
+            stat_l[st * 128 + ra] = sa;
+            stat_m[st * 128 + rb] = mb;
+            stat_l[st * 128 + rb] = sbm;
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars[C::bStFull + st]);
           ++cseg;
@@ -518,18 +538,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   } else {
     regs_set<kLaunchRegs, kRegsEpilogue>();
     // ------------------------------------------------------------ epilogue
-    const int q4 = warp - 4;
+    const int q4 = warp - kWarpEpi;
     const int r = q4 * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t opart = tmem + lane_base + C::kColOpart;
     const uint32_t otot = tmem + lane_base + C::kColOtot;
     const int D = p.D;
     uint32_t cseg = 0;
-    long long n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
+    uint32_t n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
       const uint8_t* prow = p.plan + (size_t)qt * G.P;
-      const QTile t = query_tile(G, qt);
+      const QTile t = query_tile<WIN>(G, qt);
       const int qrow = t.q0 + r;
       const bool valid = r < t.rows;
       float m_tot = kNegInf, l_tot = 0.f;
@@ -537,20 +557,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       // (1) cached states of the REUSE pairs: merged first, while the MMA and
       //     softmax warps compute the item's first fresh state
       for (int j = 0; j < G.P; ++j) {
-        const int seg = visit_seg(G, idx, j);
+        const int seg = visit_seg<WIN>(G, idx, j);
         if (prow[seg] == DT_PLAN_COMPUTE) continue;
-        if (r == 0) { n_skip += counted_blocks(G, qt, seg); ++n_read; }
-        if (G.window > 0) { use_r = true; continue; }     // complement reused: add R at the end
+        if (r == 0) { n_skip += counted_blocks<WIN>(G, qt, seg); ++n_read; }
+        if (WIN) { use_r = true; continue; }     // complement reused: add R at the end
         const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
-        const float lse_c = valid ? p.cache_L[slot] : kNegInf;
+        const float lse_c = valid ? __ldcs(p.cache_L + slot) : kNegInf;
         const bool nonempty = lse_c > kNegInf;
-        float4 cv[DP / 4];                                  // the whole cached row, loads in flight together
-        const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
-        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < DP / 4; ++c) cv[c] = (valid && 4 * c < D) ? src[c] : z4;
-#pragma unroll
-        for (int c = 0; c < DP / 4; ++c) cv[c] = nonempty ? cv[c] : z4;
         const float m_c = lse_c * kLog2e;
         float a, b, m_new;
         if (!have) { m_new = m_c; a = 0.f; b = nonempty ? 1.f : 0.f; }
@@ -560,20 +573,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           b = nonempty ? ex2(m_c - m_new) : 0.f;
         }
         const float l_new = (have ? a * l_tot : 0.f) + b;
+        const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+        for (int c1 = 0; c1 < DP; c1 += 64) {             // up to 64 cached columns in flight together
+          constexpr int kG = DP < 64 ? DP / 4 : 16;
+          float4 cv[kG];
 #pragma unroll
-        for (int c0 = 0; c0 < DP; c0 += 16) {
-          uint32_t ot[16], o16[16];
-          tmem_ld16(otot + c0, ot);
-          tmem_wait_ld();
+          for (int c = 0; c < kG; ++c)
+            cv[c] = (c1 + 4 * c < DP && valid && nonempty && c1 + 4 * c < D) ? __ldcs(src + c1 / 4 + c) : z4;
 #pragma unroll
-          for (int jj = 0; jj < 16; jj += 4) {
-            const float4 x = cv[(c0 + jj) / 4];
-            o16[jj + 0] = f2u(have ? fmaf(a, u2f(ot[jj + 0]), b * x.x) : b * x.x);
-            o16[jj + 1] = f2u(have ? fmaf(a, u2f(ot[jj + 1]), b * x.y) : b * x.y);
-            o16[jj + 2] = f2u(have ? fmaf(a, u2f(ot[jj + 2]), b * x.z) : b * x.z);
-            o16[jj + 3] = f2u(have ? fmaf(a, u2f(ot[jj + 3]), b * x.w) : b * x.w);
+          for (int c0 = c1; c0 < DP && c0 < c1 + 64; c0 += 16) {
+            uint32_t ot[16];
+            tmem_ld16(otot + c0, ot);
+            tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 16; jj += 4) {
+              const float4 x = cv[(c0 - c1 + jj) / 4];
+              ot[jj + 0] = f2u(have ? fmaf(a, u2f(ot[jj + 0]), b * x.x) : b * x.x);
+              ot[jj + 1] = f2u(have ? fmaf(a, u2f(ot[jj + 1]), b * x.y) : b * x.y);
+              ot[jj + 2] = f2u(have ? fmaf(a, u2f(ot[jj + 2]), b * x.z) : b * x.z);
+              ot[jj + 3] = f2u(have ? fmaf(a, u2f(ot[jj + 3]), b * x.w) : b * x.w);
+            }
+            tmem_st16(otot + c0, ot);
           }
-          tmem_st16(otot + c0, o16);
         }
         tmem_wait_st();
         if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
@@ -581,16 +604,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       }
       // (2) fresh states, in the order the MMA produces them
       for (int j = 0; j < G.P; ++j) {
-        const int seg = visit_seg(G, idx, j);
+        const int seg = visit_seg<WIN>(G, idx, j);
         if (prow[seg] != DT_PLAN_COMPUTE) continue;
-        const int nt = key_set(G, qt, seg).ntiles();
+        const int nt = key_set<WIN>(G, qt, seg).ntiles();
         const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
-        if (r == 0) { n_comp += counted_blocks(G, qt, seg); ++n_fresh; }
+        if (r == 0) { n_comp += counted_blocks<WIN>(G, qt, seg); ++n_fresh; }
         if (nt == 0) {             // empty key set: the identity state
-          if (G.window == 0 && valid) {
+          if (!WIN && valid) {
             float4* dst = reinterpret_cast<float4*>(p.cache_O + slot * D);
-            for (int d = 0; d < D / 4; ++d) dst[d] = make_float4(0.f, 0.f, 0.f, 0.f);
-            p.cache_L[slot] = kNegInf;
+            for (int d = 0; d < D / 4; ++d) __stcs(dst + d, make_float4(0.f, 0.f, 0.f, 0.f));
+            __stcs(p.cache_L + slot, kNegInf);
           }
           continue;
         }
@@ -610,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[C::bOFree]);
-        if (warp == 4) DT_TR(7, cseg);
+        if (warp == kWarpEpi) DT_TR(7, cseg);
         const bool nonempty = l_s > 0.f;
         const float inv_l = nonempty ? 1.f / l_s : 0.f;
         float a, b, m_new;
@@ -621,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           b = nonempty ? ex2(m_s - m_new) : 0.f;
         }
         const float l_new = (have ? a * l_tot : 0.f) + b * l_s;
-        const bool make_r = G.window > 0 && seg == 1;
+        const bool make_r = WIN && seg == 1;
         const float inv_tot = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
         const float inv_new = l_new > 0.f ? 1.f / l_new : 0.f;
 #pragma unroll
@@ -629,42 +652,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           uint32_t ot[16];
           tmem_ld16(otot + c0, ot);
           tmem_wait_ld();
-          float nw[16];
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const float x = u2f(op[c0 + jj]);
-            nw[jj] = have ? fmaf(a, u2f(ot[jj]), b * x) : b * x;
-          }
-          if (valid) {
-            if (G.window == 0) {
-              float* dst = p.cache_O + slot * D + c0;
+          for (int jj = 0; jj < 16; jj += 4) {
+            float old[4], nw[4], x[4];
 #pragma unroll
-              for (int jj = 0; jj < 16; jj += 4)
-                if (c0 + jj < D)
-                  *reinterpret_cast<float4*>(dst + jj) =
-                      make_float4(u2f(op[c0 + jj]) * inv_l, u2f(op[c0 + jj + 1]) * inv_l,
-                                  u2f(op[c0 + jj + 2]) * inv_l, u2f(op[c0 + jj + 3]) * inv_l);
-            } else if (make_r) {
-              float* dst = p.R + ((size_t)h * G.S + qrow) * D + c0;
-#pragma unroll
-              for (int jj = 0; jj < 16; jj += 4)
-                if (c0 + jj < D) {
-                  float4 v;
-                  v.x = nw[jj] * inv_new - (have ? u2f(ot[jj]) * inv_tot : 0.f);
-                  v.y = nw[jj + 1] * inv_new - (have ? u2f(ot[jj + 1]) * inv_tot : 0.f);
-                  v.z = nw[jj + 2] * inv_new - (have ? u2f(ot[jj + 2]) * inv_tot : 0.f);
-                  v.w = nw[jj + 3] * inv_new - (have ? u2f(ot[jj + 3]) * inv_tot : 0.f);
-                  *reinterpret_cast<float4*>(dst + jj) = v;
-                }
+            for (int k = 0; k < 4; ++k) {
+              old[k] = u2f(ot[jj + k]);
+              x[k] = u2f(op[c0 + jj + k]);
+              nw[k] = have ? fmaf(a, old[k], b * x[k]) : b * x[k];
+              ot[jj + k] = f2u(nw[k]);
+            }
+            if (valid && c0 + jj < D) {
+              if (!WIN) {
+                __stcs(reinterpret_cast<float4*>(p.cache_O + slot * D + c0 + jj),
+                       make_float4(x[0] * inv_l, x[1] * inv_l, x[2] * inv_l, x[3] * inv_l));
+              } else if (make_r) {
+                float4 v;
+                v.x = nw[0] * inv_new - (have ? old[0] * inv_tot : 0.f);
+                v.y = nw[1] * inv_new - (have ? old[1] * inv_tot : 0.f);
+                v.z = nw[2] * inv_new - (have ? old[2] * inv_tot : 0.f);
+                v.w = nw[3] * inv_new - (have ? old[3] * inv_tot : 0.f);
+                __stcs(reinterpret_cast<float4*>(p.R + ((size_t)h * G.S + qrow) * D + c0 + jj), v);
+              }
             }
           }
-          uint32_t o16[16];
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) o16[jj] = f2u(nw[jj]);
-          tmem_st16(otot + c0, o16);
+          tmem_st16(otot + c0, ot);
         }
         tmem_wait_st();
-        if (G.window == 0 && valid) p.cache_L[slot] = nonempty ? (m_s + lg2(l_s)) * kLn2 : kNegInf;
+        if (!WIN && valid) __stcs(p.cache_L + slot, nonempty ? (m_s + lg2(l_s)) * kLn2 : kNegInf);
         if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
         have = have || nonempty;
         ++cseg;
@@ -686,18 +701,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
                 float v0 = have ? u2f(ot[j]) * inv : 0.f, v1 = have ? u2f(ot[j + 1]) * inv : 0.f;
                 float v2 = have ? u2f(ot[j + 2]) * inv : 0.f, v3 = have ? u2f(ot[j + 3]) * inv : 0.f;
                 if (use_r) {
-                  const float4 rv = *reinterpret_cast<const float4*>(rr + c0 + j);
+                  const float4 rv = __ldcs(reinterpret_cast<const float4*>(rr + c0 + j));
                   v0 += rv.x; v1 += rv.y; v2 += rv.z; v3 += rv.w;
                 }
                 uint2 pk;
                 pk.x = pack_bf16x2(v0, v1);
                 pk.y = pack_bf16x2(v2, v3);
-                *reinterpret_cast<uint2*>(dst + c0 + j) = pk;
+                __stcs(reinterpret_cast<uint2*>(dst + c0 + j), pk);
               }
             }
           }
         }
-        if (valid) p.L[(size_t)h * G.S + qrow] = (have && l_tot > 0.f) ? (m_tot + lg2(l_tot)) * kLn2 : kNegInf;
+        if (valid) __stcs(p.L + (size_t)h * G.S + qrow, (have && l_tot > 0.f) ? (m_tot + lg2(l_tot)) * kLn2 : kNegInf);
       }
     }
   ep_done:
@@ -711,23 +726,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-template <int DP>
+template <int DP, bool WIN>
 int launch_dp(const AttnParams& kp, int grid, cudaStream_t stream) {
   using C = Cfg<DP>;
   static bool attr_set = false;   // per-process; the attribute is per device function
   if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_partial_fused_kernel<DP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_partial_fused_kernel<DP, WIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmem) != cudaSuccess)
       return DT_ERR_CUDA;
     attr_set = true;
   }
-  attn_partial_fused_kernel<DP><<<grid, kThreads, C::kSmem, stream>>>(kp);
+  attn_partial_fused_kernel<DP, WIN><<<grid, kThreads, C::kSmem, stream>>>(kp);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
 }
 
@@ -750,9 +765,10 @@ int attn_fused_smem_bytes(int dp) {
 
 int launch_attn_fused(const AttnParams& kp, int dp, int grid, cudaStream_t stream) {
   switch (dp) {
-    case 64: return launch_dp<64>(kp, grid, stream);
-    case 80: return launch_dp<80>(kp, grid, stream);
-    case 128: return launch_dp<128>(kp, grid, stream);
+    case 64: return kp.window > 0 ? launch_dp<64, true>(kp, grid, stream) : launch_dp<64, false>(kp, grid, stream);
+    case 80: return kp.window > 0 ? launch_dp<80, true>(kp, grid, stream) : launch_dp<80, false>(kp, grid, stream);
+    case 128:
+      return kp.window > 0 ? launch_dp<128, true>(kp, grid, stream) : launch_dp<128, false>(kp, grid, stream);
   }
   return DT_ERR_UNSUPPORTED;
 }

@@ -68,15 +68,22 @@ DT_HD Geom make_geom(int H, int S, int D, int P, int window) {
   return g;
 }
 
+// Mode of a geometry call: W = 0 partition mode, 1 window mode, -1 read from
+// g.window at run time.  Kernels instantiate the mode they run so that the
+// other mode's code is not compiled into them.
+template <int W>
+DT_HD bool is_window(const Geom& g) { return W < 0 ? g.window > 0 : W == 1; }
+
 DT_HD int part_begin(const Geom& g, int k) { return imin(k * g.c, g.S); }
 DT_HD int part_end(const Geom& g, int k) { return imin((k + 1) * g.c, g.S); }
 
 // Query tile qt -> (partition, first row, rows).
 struct QTile { int part, q0, rows; };
 
+template <int W = -1>
 DT_HD QTile query_tile(const Geom& g, int qt) {
   QTile t;
-  if (g.window > 0) {
+  if (is_window<W>(g)) {
     t.part = 0;
     t.q0 = qt * kTile;
     t.rows = imin(kTile, g.S - t.q0);
@@ -111,16 +118,17 @@ struct KeySet {
   DT_HD int tile(int i) const { return i < (r0e - r0b) ? r0b + i : r1b + (i - (r0e - r0b)); }
 };
 
+template <int W = -1>
 DT_HD KeySet key_set(const Geom& g, int qt, int seg) {
   KeySet ks;
-  if (g.window == 0) {
+  if (!is_window<W>(g)) {
     ks.base = part_begin(g, seg);
     ks.kend = part_end(g, seg);
     ks.r0b = 0; ks.r0e = ceil_div(ks.kend - ks.base, kTile);
     ks.r1b = ks.r1e = 0;
     return ks;
   }
-  QTile t = query_tile(g, qt);
+  QTile t = query_tile<W>(g, qt);
   int q0 = t.q0, q1 = t.q0 + t.rows - 1;
   ks.base = 0; ks.kend = g.S;
   // touching range [lo, hi] and fully-inside range [fi, fl] (may be empty)
@@ -144,10 +152,11 @@ DT_HD KeySet key_set(const Geom& g, int qt, int seg) {
 // Distinct 128x128 blocks of key set `seg` of query tile `qt` that count as
 // "computed" (or "skipped") blocks: in window mode the straddling tiles are
 // counted once, in the window set.
+template <int W = -1>
 DT_HD int counted_blocks(const Geom& g, int qt, int seg) {
-  KeySet ks = key_set(g, qt, seg);
-  if (g.window == 0 || seg == 0) return ks.ntiles();
-  QTile t = query_tile(g, qt);
+  KeySet ks = key_set<W>(g, qt, seg);
+  if (!is_window<W>(g) || seg == 0) return ks.ntiles();
+  QTile t = query_tile<W>(g, qt);
   int q0 = t.q0, q1 = t.q0 + t.rows - 1, n = 0;
   for (int i = 0; i < ks.ntiles(); ++i)
     if (!wtile_touches(g, q0, q1, ks.tile(i))) ++n;
