@@ -85,7 +85,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when t
 // Timeline tracing for kernel development (compiled only with -DDT_TRACE):
 // CTA 0 records clock64 stamps of each role into a caller-provided buffer.
 #ifdef DT_TRACE
-__device__ uint64_t* g_dt_trace = nullptr;
+__constant__ uint64_t* g_dt_trace = nullptr;   // constant bank: no global load per stamp
 #define DT_TR(ev, idx)                                                                             \
   do {                                                                                             \
     if (blockIdx.x == 0 && (threadIdx.x & 31) == 0 && g_dt_trace && (idx) < 4096)                 \
@@ -172,23 +172,30 @@ __device__ __forceinline__ bool issue_pv(uint64_t* bars, uint32_t tmem, uint32_t
   if (!mbar_wait(&bars[C::bVFull + st], (g / C::kStages) & 1, abort, status, DT_ERR_TIMEOUT, lim)) return false;
   DT_TR(5, g);
   tc_fence_after();
-  const uint32_t aP = tmem + C::kColS + sb * 128;
+  uint32_t aP = tmem + C::kColS + sb * 128;
   const uint32_t vb = aV + st * C::kTileBytes;
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {          // 16 keys per MMA
-    const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-    const uint64_t vd = smem_desc(vb + kk * 2048, C::kBlk, 1024, kSwizzle128B);
-    const uint64_t vdt = smem_desc(vb + C::kN64 * C::kBlk + kk * 512, C::kTailBytes, 256, kSwizzle32B);
-    mma_ts(tmem + C::kColOpart, aP + kk * 8, vd, idesc_pv, acc);
-    if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + kk * 8, vdt, idesc_pvt, acc);
+  // 16 keys per MMA; descriptors advance by 16 V rows (2048 bytes in the
+  // 128-byte-swizzled blocks, 512 in the 32-byte-swizzled tail)
+  uint64_t vd = smem_desc(vb, C::kBlk, 1024, kSwizzle128B);
+  uint64_t vdt = smem_desc(vb + C::kN64 * C::kBlk, C::kTailBytes, 256, kSwizzle32B);
+  uint32_t acc = first ? 0u : 1u;
+#pragma unroll 1
+  for (int kk = 0; kk < 8; ++kk) {
+    mma_ts(tmem + C::kColOpart, aP, vd, idesc_pv, acc);
+    if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP, vdt, idesc_pvt, acc);
     if (precise) {                          // P = P_hi + P_lo (P_lo in columns 64..127)
-      mma_ts(tmem + C::kColOpart, aP + 64 + kk * 8, vd, idesc_pv, 1u);
-      if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + 64 + kk * 8, vdt, idesc_pvt, 1u);
+      mma_ts(tmem + C::kColOpart, aP + 64, vd, idesc_pv, 1u);
+      if (C::kTail) mma_ts(tmem + C::kColOpart + 64 * C::kN64, aP + 64, vdt, idesc_pvt, 1u);
     }
+    acc = 1u;
+    aP += 8;
+    vd += 2048 >> 4;
+    vdt += 512 >> 4;
   }
   mma_commit(&bars[C::bVEmpty + st]);
   mma_commit(&bars[C::bODone]);
   if (last) mma_commit(&bars[C::bODSeg]);
+  DT_TR(12, g);
   return true;
 }
 
@@ -333,14 +340,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               ok = false;
               break;
             }
+            DT_TR(11, g);
             tc_fence_after();
             const uint32_t dS = tmem + C::kColS + (g & 1) * 128;
             const uint32_t kb = aK + st * C::kTileBytes;
+            // 16 head-dim columns (32 bytes of each swizzled row) per MMA
+            uint32_t acc = 0u;
+#pragma unroll 1
+            for (int blk = 0; blk < C::kN64; ++blk) {
+              uint64_t qd = smem_desc(aQ + blk * C::kBlk, 16, 1024, kSwizzle128B);
+              uint64_t kd = smem_desc(kb + blk * C::kBlk, 16, 1024, kSwizzle128B);
 #pragma unroll
-            for (int kk = 0; kk < 4 * C::kN64; ++kk) {      // 16 head-dim columns per MMA
-              const uint32_t off = (kk >> 2) * C::kBlk + (kk & 3) * 32;
-              mma_ss(dS, smem_desc(aQ + off, 16, 1024, kSwizzle128B), smem_desc(kb + off, 16, 1024, kSwizzle128B),
-                     idesc_qk, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk) {
+                mma_ss(dS, qd, kd, idesc_qk, acc);
+                acc = 1u;
+                qd += 32 >> 4;
+                kd += 32 >> 4;
+              }
             }
             if (C::kTail) {
               const uint32_t off = C::kN64 * C::kBlk;
@@ -543,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t opart = tmem + lane_base + C::kColOpart;
     const uint32_t otot = tmem + lane_base + C::kColOtot;
-    const int D = p.D;
+    constexpr int D = DP == 80 ? 72 : DP;   // head dims 64, 72, 128 (padded 64, 80, 128)
     uint32_t cseg = 0;
     uint32_t n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
@@ -554,6 +570,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const bool valid = r < t.rows;
       float m_tot = kNegInf, l_tot = 0.f;
       bool have = false, use_r = false;
+      {   // O_tot starts at zero, so the merges below need no separate first-state case
+        uint32_t z[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) z[k] = 0u;
+#pragma unroll 1
+        for (int c0 = 0; c0 < DP; c0 += 16) tmem_st16(otot + c0, z);
+        tmem_wait_st();
+      }
       // (1) cached states of the REUSE pairs: merged first, while the MMA and
       //     softmax warps compute the item's first fresh state
       for (int j = 0; j < G.P; ++j) {
@@ -572,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           a = ex2(m_tot - m_new);
           b = nonempty ? ex2(m_c - m_new) : 0.f;
         }
-        const float l_new = (have ? a * l_tot : 0.f) + b;
+        const float l_new = a * l_tot + b;
         const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
         const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
@@ -590,10 +614,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 #pragma unroll
             for (int jj = 0; jj < 16; jj += 4) {
               const float4 x = cv[(c0 - c1 + jj) / 4];
-              ot[jj + 0] = f2u(have ? fmaf(a, u2f(ot[jj + 0]), b * x.x) : b * x.x);
-              ot[jj + 1] = f2u(have ? fmaf(a, u2f(ot[jj + 1]), b * x.y) : b * x.y);
-              ot[jj + 2] = f2u(have ? fmaf(a, u2f(ot[jj + 2]), b * x.z) : b * x.z);
-              ot[jj + 3] = f2u(have ? fmaf(a, u2f(ot[jj + 3]), b * x.w) : b * x.w);
+              ot[jj + 0] = f2u(fmaf(a, u2f(ot[jj + 0]), b * x.x));
+              ot[jj + 1] = f2u(fmaf(a, u2f(ot[jj + 1]), b * x.y));
+              ot[jj + 2] = f2u(fmaf(a, u2f(ot[jj + 2]), b * x.z));
+              ot[jj + 3] = f2u(fmaf(a, u2f(ot[jj + 3]), b * x.w));
             }
             tmem_st16(otot + c0, ot);
           }
@@ -643,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           a = ex2(m_tot - m_new);
           b = nonempty ? ex2(m_s - m_new) : 0.f;
         }
-        const float l_new = (have ? a * l_tot : 0.f) + b * l_s;
+        const float l_new = a * l_tot + b * l_s;
         const bool make_r = WIN && seg == 1;
         const float inv_tot = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
         const float inv_new = l_new > 0.f ? 1.f / l_new : 0.f;
@@ -659,7 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             for (int k = 0; k < 4; ++k) {
               old[k] = u2f(ot[jj + k]);
               x[k] = u2f(op[c0 + jj + k]);
-              nw[k] = have ? fmaf(a, old[k], b * x[k]) : b * x[k];
+              nw[k] = fmaf(a, old[k], b * x[k]);
               ot[jj + k] = f2u(nw[k]);
             }
             if (valid && c0 + jj < D) {
@@ -668,10 +692,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
                        make_float4(x[0] * inv_l, x[1] * inv_l, x[2] * inv_l, x[3] * inv_l));
               } else if (make_r) {
                 float4 v;
-                v.x = nw[0] * inv_new - (have ? old[0] * inv_tot : 0.f);
-                v.y = nw[1] * inv_new - (have ? old[1] * inv_tot : 0.f);
-                v.z = nw[2] * inv_new - (have ? old[2] * inv_tot : 0.f);
-                v.w = nw[3] * inv_new - (have ? old[3] * inv_tot : 0.f);
+                v.x = nw[0] * inv_new - old[0] * inv_tot;
+                v.y = nw[1] * inv_new - old[1] * inv_tot;
+                v.z = nw[2] * inv_new - old[2] * inv_tot;
+                v.w = nw[3] * inv_new - old[3] * inv_tot;
                 __stcs(reinterpret_cast<float4*>(p.R + ((size_t)h * G.S + qrow) * D + c0 + jj), v);
               }
             }
@@ -698,8 +722,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 #pragma unroll
             for (int j = 0; j < 16; j += 4) {
               if (c0 + j < D) {
-                float v0 = have ? u2f(ot[j]) * inv : 0.f, v1 = have ? u2f(ot[j + 1]) * inv : 0.f;
-                float v2 = have ? u2f(ot[j + 2]) * inv : 0.f, v3 = have ? u2f(ot[j + 3]) * inv : 0.f;
+                float v0 = u2f(ot[j]) * inv, v1 = u2f(ot[j + 1]) * inv;
+                float v2 = u2f(ot[j + 2]) * inv, v3 = u2f(ot[j + 3]) * inv;
                 if (use_r) {
                   const float4 rv = __ldcs(reinterpret_cast<const float4*>(rr + c0 + j));
                   v0 += rv.x; v1 += rv.y; v2 += rv.z; v3 += rv.w;
