@@ -66,6 +66,23 @@ def peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of ``values`` over all ranks of the default process
+    group (the identity on one rank).  Every multi-rank time is taken this way."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(flops_per_rank, world, ms):
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's time."""
+    return flops_per_rank * world / (ms * 1e-3) / 1e12
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for fn in ("attn_fused_sm100.cu", "sm100.cuh", "geometry.h", "attn_fused.h"):
@@ -290,10 +307,7 @@ def main():
         sess.check()
         total_ms = t0.elapsed_time(t1)
         kern_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
-        if world > 1:
-            t = torch.tensor([total_ms, kern_ms], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            total_ms, kern_ms = float(t[0]), float(t[1])
+        total_ms, kern_ms = max_over_ranks([total_ms, kern_ms], "cuda")
         return total_ms / n_steps, kern_ms, counts
 
     # headline
@@ -301,7 +315,7 @@ def main():
         ms_step, kern_ms, counts = timed(args.steps, args.warmup, r)
     clocks = clk.summary()
     flops = counts["computed_flops"]
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = job_throughput(flops, world, ms_step)
     pk, pk_kind = peaks()
     peak_tf = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (kern_ms * 1e-3) / 1e12
@@ -366,14 +380,10 @@ def main():
             e2e_step()
         b.record(cur)
         barrier()
-        ems = a.elapsed_time(b) / ke
-        if world > 1:
-            t = torch.tensor([ems], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t[0])
+        ems = max_over_ranks([a.elapsed_time(b) / ke], "cuda")[0]
         h2d = sum(x.numel() * x.element_size() for x in hq) + sess.nqt * sess.nseg
         d2h = ho.numel() * 2 + hl.numel() * 4
-        e2e = {"value": flops * world / (ems * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ems,
+        e2e = {"value": job_throughput(flops, world, ems), "unit": "TFLOP/s", "ms_per_step": ems,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     cpu = None
