@@ -31,12 +31,14 @@
 //                         key set: O_part (TMEM) -> registers (O_part released at
 //                         once) -> normalised fresh state -> cache slot, composed
 //                         into O_tot; per item: O_tot -> O (bf16), LSE
-//   warp 12     MMA:      tcgen05.mma S = Q K^T (smem x smem), O_part += P V
-//                         (P from TMEM, V from smem); TMEM alloc/free
+//   warp 12     MMA QK:   tcgen05.mma S = Q K^T (smem x smem); TMEM alloc/free
+//   warp 15     MMA PV:   tcgen05.mma O_part += P V (P from TMEM, V from smem).
+//                         Two issuing threads, because one thread issues an
+//                         MMA only every ~50 clk: 16 MMAs per 128x128 tile
+//                         would nearly fill a single issuer's time.
 //   warp 13     TMA:      Q once per item, K tiles into an NS-stage ring
 //   warp 14     TMA:      V tiles into an NS-stage ring (released separately
 //                         from K: a K stage frees as soon as its QK^T is done)
-//   warp 15     idle (completes the fourth warpgroup)
 // Tensor memory (512 columns): S/P double buffer [0,256), O_part [256,256+DP),
 // O_tot [256+DP, 256+2*DP).  DP = head dim padded to a multiple of 16 (72 -> 80):
 // a 64-column block uses the 128-byte swizzle, the 16-column tail of D=72 the
@@ -66,9 +68,9 @@ namespace {
 
 using namespace sm100;
 
-// 4 warpgroups: softmax (warps 0-7), epilogue (8-11), MMA (12) + TMA (13, 14) + idle (15).
+// 4 warpgroups: softmax (warps 0-7), epilogue (8-11), MMA QK (12) + TMA (13, 14) + MMA PV (15).
 constexpr int kThreads = 512;
-constexpr int kWarpEpi = 8, kWarpMma = 12, kWarpTmaK = 13, kWarpTmaV = 14;
+constexpr int kWarpEpi = 8, kWarpMma = 12, kWarpTmaK = 13, kWarpTmaV = 14, kWarpMmaPV = 15;
 // Registers per thread at launch (ptxas: 65536 / 512; the build checks it) and
 // the per-warpgroup split after setmaxnreg.  The split must fit the launch
 // pool: 128 * (2 * kRegsSoftmax + kRegsEpilogue + kRegsOther) <= kThreads * kLaunchRegs.
@@ -111,8 +113,8 @@ struct Cfg {
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = 1, bKFull = 2, bVFull = 2 + kStages, bKEmpty = 2 + 2 * kStages,
                        bVEmpty = 2 + 3 * kStages, bSFull = 2 + 4 * kStages, bPFull = bSFull + 2,
-                       bODone = bPFull + 2, bODSeg = bODone + 1, bOFree = bODSeg + 1, bStFull = bOFree + 1,
-                       bStFree = bStFull + 2, bDrain = bStFree + 2, kNumBars = bDrain + 1;
+                       bPVDone = bPFull + 2, bODSeg = bPVDone + 2, bOFree = bODSeg + 1, bStFull = bOFree + 1,
+                       bStFree = bStFull + 2, bDrain = bStFree + 2, bDrainPV = bDrain + 1, kNumBars = bDrainPV + 1;
   static constexpr int kStatsBytes = 2 * 2 * 128 * 4;
   static constexpr int kSmem = kTileBytes * (1 + 2 * kStages) + kStatsBytes + kNumBars * 8 + 16;
 };
@@ -193,7 +195,7 @@ __device__ __forceinline__ bool issue_pv(uint64_t* bars, uint32_t tmem, uint32_t
     vdt += 512 >> 4;
   }
   mma_commit(&bars[C::bVEmpty + st]);
-  mma_commit(&bars[C::bODone]);
+  mma_commit(&bars[C::bPVDone + sb]);
   if (last) mma_commit(&bars[C::bODSeg]);
   DT_TR(12, g);
   return true;
@@ -314,12 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      uint32_t g = 0, nq = 0, cseg = 0;
-      // the PV of the newest tile is issued after the next tile's QK^T
-      int pv_valid = 0, pv_first = 0, pv_last = 0, pv_precise = 0;
-      uint32_t pv_g = 0, pv_seg = 0;
+      uint32_t g = 0, nq = 0;
       bool ok = true;
-
 
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
@@ -337,6 +335,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             const int st = g % C::kStages;
             DT_TR(10, g);
             if (!mbar_wait(&bars[C::bKFull + st], (g / C::kStages) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) {
+              ok = false;
+              break;
+            }
+            // S buffer g&1 held P(g-2): its PV (issued by the PV warp) must be done
+            if (g >= 2 && !mbar_wait(&bars[C::bPVDone + (g & 1)], ((g - 2) >> 1) & 1, abort_flag, p.status,
+                                     DT_ERR_TIMEOUT, lim)) {
               ok = false;
               break;
             }
@@ -366,24 +370,43 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             mma_commit(&bars[C::bSFull + (g & 1)]);
             mma_commit(&bars[C::bKEmpty + st]);
             DT_TR(0, g);
-            if (pv_valid && !issue_pv<DP>(bars, tmem, aV, pv_g, pv_seg, pv_first, pv_last, pv_precise, abort_flag,
-                                          p.status, lim)) {
-              ok = false;
-              break;
-            }
-            pv_valid = 1; pv_g = g; pv_first = (i == 0); pv_last = (i == nt - 1); pv_seg = cseg;
-            pv_precise = (WIN && seg == 0);
           }
-          ++cseg;
         }
         mma_commit(&bars[C::bQEmpty]);
       }
-      if (ok && pv_valid)
-        issue_pv<DP>(bars, tmem, aV, pv_g, pv_seg, pv_first, pv_last, pv_precise, abort_flag, p.status, lim);
-      // all MMAs of this CTA complete before tensor memory is freed
+      // all MMAs this thread issued complete before tensor memory is freed
       mma_commit(&bars[C::bDrain]);
       volatile int never = 0;
       mbar_wait(&bars[C::bDrain], 0, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
+    }
+    __syncwarp();
+   } else if (warp == kWarpMmaPV) {
+    // ------------------------------------------------------------ PV issuer
+    // A second issuing thread: one thread issues a tcgen05.mma only every ~50
+    // clk, so QK^T and PV come from separate warps.  Their ordering is explicit:
+    // PV(g) waits for P(g); QK^T(g+2) waits for PV(g) through bPVDone.
+    if (lane == 0) {
+      const uint32_t aV = smem_u32(sV);
+      uint32_t g = 0, cseg = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+        const int qt = idx - (idx / G.nqt) * G.nqt;
+        const uint8_t* prow = p.plan + (size_t)qt * G.P;
+        if (!item_has_compute<WIN>(G, qt, prow)) continue;
+        for (int j = 0; j < G.P && ok; ++j) {
+          const int seg = visit_seg<WIN>(G, idx, j);
+          if (prow[seg] != DT_PLAN_COMPUTE) continue;
+          const int nt = key_set<WIN>(G, qt, seg).ntiles();
+          if (nt == 0) continue;
+          for (int i = 0; i < nt && ok; ++i, ++g)
+            ok = issue_pv<DP>(bars, tmem, aV, g, cseg, i == 0, i == nt - 1, WIN && seg == 0, abort_flag, p.status,
+                              lim);
+          ++cseg;
+        }
+      }
+      mma_commit(&bars[C::bDrainPV]);
+      volatile int never = 0;
+      mbar_wait(&bars[C::bDrainPV], 0, &never, p.status, DT_ERR_TIMEOUT, kDrainLimitNs);
     }
     __syncwarp();
    }
@@ -471,7 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           const bool resa = (i > 0) && (na != ma), resb = (i > 0) && (nb != mb);
           if (__any_sync(0xffffffffu, resa || resb)) {
             // O_part holds the previous tiles' sum: wait for its last PV, then rescale
-            if (!warp_wait(&bars[C::bODone], (g - 1) & 1, abort_flag, p.status, lim)) goto sm_done;
+            if (!warp_wait(&bars[C::bPVDone + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag, p.status, lim))
+              goto sm_done;
             tc_fence_after();
             const float alpha_a = resa ? ex2(ma - na) : 1.f, alpha_b = resb ? ex2(mb - nb) : 1.f;
             const uint32_t oc = tmem + lane_base + C::kColOpart;
