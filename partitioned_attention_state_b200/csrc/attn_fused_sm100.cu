@@ -27,10 +27,11 @@
 //                         exponential unit busy while the other warp loads S,
 //                         reduces its max or stores P.
 //   warps 8-11  epilogue: per reused key set (first, off the critical path):
-//                         cached state composed into O_tot (TMEM); per computed
-//                         key set: O_part (TMEM) -> registers (O_part released at
-//                         once) -> normalised fresh state -> cache slot, composed
-//                         into O_tot; per item: O_tot -> O (bf16), LSE
+//                         cached state composed into O_tot (shared memory); per
+//                         computed key set: O_part (TMEM) -> registers (O_part
+//                         released at once) -> normalised fresh state -> cache
+//                         slot, composed into O_tot; per item: O_tot -> O
+//                         (bf16), LSE
 //   warp 12     MMA QK:   tcgen05.mma S = Q K^T (smem x smem); TMEM alloc/free
 //   warp 15     MMA PV:   tcgen05.mma O_part += P V (P from TMEM, V from smem).
 //                         Two issuing threads, because one thread issues an
@@ -39,8 +40,11 @@
 //   warp 13     TMA:      Q once per item, K tiles into an NS-stage ring
 //   warp 14     TMA:      V tiles into an NS-stage ring (released separately
 //                         from K: a K stage frees as soon as its QK^T is done)
-// Tensor memory (512 columns): S/P double buffer [0,256), O_part [256,256+DP),
-// O_tot [256+DP, 256+2*DP).  DP = head dim padded to a multiple of 16 (72 -> 80):
+// Tensor memory (512 columns): three S/P buffers [0,384), O_part [384,384+DP).
+// Three buffers let QK^T(g+3) wait only for PV(g), so the chain
+// P(g) -> PV(g) -> QK^T(g+3) -> softmax spans three tiles.  O_tot (the
+// running composition of an item's states) lives in shared memory, column-
+// major fp32, one row per epilogue thread.  DP = head dim padded to a multiple of 16 (72 -> 80):
 // a 64-column block uses the 128-byte swizzle, the 16-column tail of D=72 the
 // 32-byte swizzle (zero-filled by TMA out-of-bounds handling).
 //
@@ -105,18 +109,20 @@ struct Cfg {
   static constexpr int kBlk = 128 * 64 * 2;            // bytes of a 128x64 bf16 block
   static constexpr int kTailBytes = 128 * 16 * 2;      // bytes of a 128x16 bf16 block
   static constexpr int kTileBytes = kN64 * kBlk + kTail * kTailBytes;   // = 128 * DP * 2
-  static constexpr int kStages = DP == 128 ? 3 : (DP == 80 ? 5 : 6);
+  static constexpr int kStages = DP == 128 ? 2 : (DP == 80 ? 4 : 5);
+  static constexpr int kNS = 3;                        // S/P buffers in tensor memory
   static constexpr int kColS = 0;
-  static constexpr int kColOpart = 256;
-  static constexpr int kColOtot = 256 + DP;
-  static_assert(kColOtot + DP <= 512, "tensor memory budget");
+  static constexpr int kColOpart = 128 * kNS;
+  static_assert(kColOpart + DP <= 512, "tensor memory budget");
+  static constexpr int kOtotBytes = DP * 128 * 4;      // O_tot in shared memory, column-major [DP][128] fp32
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = 1, bKFull = 2, bVFull = 2 + kStages, bKEmpty = 2 + 2 * kStages,
-                       bVEmpty = 2 + 3 * kStages, bSFull = 2 + 4 * kStages, bPFull = bSFull + 2,
-                       bPVDone = bPFull + 2, bODSeg = bPVDone + 2, bOFree = bODSeg + 1, bStFull = bOFree + 1,
+                       bVEmpty = 2 + 3 * kStages, bSFull = 2 + 4 * kStages, bPFull = bSFull + kNS,
+                       bPVDone = bPFull + kNS, bODSeg = bPVDone + kNS, bOFree = bODSeg + 1, bStFull = bOFree + 1,
                        bStFree = bStFull + 2, bDrain = bStFree + 2, bDrainPV = bDrain + 1, kNumBars = bDrainPV + 1;
   static constexpr int kStatsBytes = 2 * 2 * 128 * 4;
-  static constexpr int kSmem = kTileBytes * (1 + 2 * kStages) + kStatsBytes + kNumBars * 8 + 16;
+  static constexpr int kSmem = kTileBytes * (1 + 2 * kStages) + kOtotBytes + kStatsBytes + kNumBars * 8 + 16;
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 // Exponentials of an unmasked tile: when kEmuMod > 0 every kEmuMod-th
@@ -126,14 +132,12 @@ constexpr int kEmuMod = 0;
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
-// Warp-level wait: lane 0 polls, the verdict is broadcast to the warp.
+// Warp-level wait: every lane checks the barrier itself (uniform control
+// flow; a lane-0 poll plus broadcast costs a few hundred cycles per wait).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status,
                                           uint64_t limit) {
-  int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status, DT_ERR_TIMEOUT, limit) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
+  const bool ok = mbar_wait(bar, parity, abort, status, DT_ERR_TIMEOUT, limit);
+  return __all_sync(0xffffffffu, ok);
 }
 
 template <bool WIN>
@@ -166,8 +170,8 @@ __device__ __forceinline__ bool issue_pv(uint64_t* bars, uint32_t tmem, uint32_t
   using C = Cfg<DP>;
   constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 64 * C::kN64, 0, 1);
   constexpr uint32_t idesc_pvt = idesc_bf16_f32(128, 16, 0, 1);
-  const uint32_t sb = g & 1;
-  if (!mbar_wait(&bars[C::bPFull + sb], (g >> 1) & 1, abort, status, DT_ERR_TIMEOUT, lim)) return false;
+  const uint32_t sb = g % C::kNS;
+  if (!mbar_wait(&bars[C::bPFull + sb], (g / C::kNS) & 1, abort, status, DT_ERR_TIMEOUT, lim)) return false;
   if (first && seg > 0 && !mbar_wait(&bars[C::bOFree], (seg - 1) & 1, abort, status, DT_ERR_TIMEOUT, lim))
     return false;
   const int st = g % C::kStages;
@@ -212,7 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   uint8_t* sQ = smem;
   uint8_t* sK = smem + C::kTileBytes;
   uint8_t* sV = sK + C::kStages * C::kTileBytes;
-  float* stat_m = reinterpret_cast<float*>(sV + C::kStages * C::kTileBytes);   // [2][128]
+  float* sO = reinterpret_cast<float*>(sV + C::kStages * C::kTileBytes);       // O_tot [DP][128]
+  float* stat_m = sO + DP * 128;                                               // [2][128]
   float* stat_l = stat_m + 256;                                                // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(stat_l + 256);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
@@ -224,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 
   if (warp == kWarpTmaK && lane == 0) {
     for (int i = 0; i < C::kNumBars; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < C::kNS; ++i) mbar_init(&bars[C::bPFull + i], 8 * 32);   // every softmax thread arrives
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[C::bPFull + i], 8);     // one arrival per softmax warp
       mbar_init(&bars[C::bStFull + i], 8);
       mbar_init(&bars[C::bStFree + i], 4);    // one arrival per epilogue warp
     }
@@ -338,15 +343,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               ok = false;
               break;
             }
-            // S buffer g&1 held P(g-2): its PV (issued by the PV warp) must be done
-            if (g >= 2 && !mbar_wait(&bars[C::bPVDone + (g & 1)], ((g - 2) >> 1) & 1, abort_flag, p.status,
-                                     DT_ERR_TIMEOUT, lim)) {
+            // S buffer g%3 held P(g-3): its PV (issued by the PV warp) must be done
+            if (g >= (uint32_t)C::kNS &&
+                !mbar_wait(&bars[C::bPVDone + g % C::kNS], (g / C::kNS - 1) & 1, abort_flag, p.status,
+                           DT_ERR_TIMEOUT, lim)) {
               ok = false;
               break;
             }
             DT_TR(11, g);
             tc_fence_after();
-            const uint32_t dS = tmem + C::kColS + (g & 1) * 128;
+            const uint32_t dS = tmem + C::kColS + (g % C::kNS) * 128;
             const uint32_t kb = aK + st * C::kTileBytes;
             // 16 head-dim columns (32 bytes of each swizzled row) per MMA
             uint32_t acc = 0u;
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               mma_ss(dS, smem_desc(aQ + off, 16, 256, kSwizzle32B), smem_desc(kb + off, 16, 256, kSwizzle32B),
                      idesc_qk, 1u);
             }
-            mma_commit(&bars[C::bSFull + (g & 1)]);
+            mma_commit(&bars[C::bSFull + g % C::kNS]);
             mma_commit(&bars[C::bKEmpty + st]);
             DT_TR(0, g);
           }
@@ -441,9 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         float la[4] = {0.f, 0.f, 0.f, 0.f}, lb[4] = {0.f, 0.f, 0.f, 0.f};
         const bool precise = WIN && seg == 0;
         for (int i = 0; i < nt; ++i, ++g) {
-          const uint32_t sb = g & 1;
-          if (!warp_wait(&bars[C::bSFull + sb], (g >> 1) & 1, abort_flag, p.status, lim)) goto sm_done;
+          const uint32_t sb = g % C::kNS;
+          if (warp == 0) DT_TR(15, g);
+          if (!warp_wait(&bars[C::bSFull + sb], (g / C::kNS) & 1, abort_flag, p.status, lim)) goto sm_done;
           if (warp == 0) DT_TR(2, g);
+          if (warp == 7) DT_TR(14, g);
           tc_fence_after();
           const int tile = visit_tile(ks, nt, idx, seg, i);
           const int k0 = ks.base + tile * kTile;
@@ -494,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           const bool resa = (i > 0) && (na != ma), resb = (i > 0) && (nb != mb);
           if (__any_sync(0xffffffffu, resa || resb)) {
             // O_part holds the previous tiles' sum: wait for its last PV, then rescale
-            if (!warp_wait(&bars[C::bPVDone + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag, p.status, lim))
+            if (!warp_wait(&bars[C::bPVDone + (g - 1) % C::kNS], ((g - 1) / C::kNS) & 1, abort_flag, p.status, lim))
               goto sm_done;
             tc_fence_after();
             const float alpha_a = resa ? ex2(ma - na) : 1.f, alpha_b = resb ? ex2(mb - nb) : 1.f;
@@ -549,9 +557,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           if (warp == 0) DT_TR(6, g);
           tmem_wait_st();
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[C::bPFull + sb]);
+          mbar_arrive(&bars[C::bPFull + sb]);      // all lanes: no divergent single-lane branch per tile
           if (warp == 0) DT_TR(4, g);
+          if (warp == 7) DT_TR(13, g);
         }
         {
           float sa = ((la[0] + la[1]) + (la[2] + la[3])), sbm = ((lb[0] + lb[1]) + (lb[2] + lb[3]));
@@ -582,8 +590,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     const int r = q4 * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t opart = tmem + lane_base + C::kColOpart;
-    const uint32_t otot = tmem + lane_base + C::kColOtot;
     constexpr int D = DP == 80 ? 72 : DP;   // head dims 64, 72, 128 (padded 64, 80, 128)
+    // O_tot of this thread's row lives in shared memory, column-major
+    // ([column][row]: consecutive threads, consecutive banks), unnormalised
+    // relative to m_tot.  Only this thread touches its row.
+    float* orow = sO + r;
     uint32_t cseg = 0;
     uint32_t n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
@@ -594,14 +605,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const bool valid = r < t.rows;
       float m_tot = kNegInf, l_tot = 0.f;
       bool have = false, use_r = false;
-      {   // O_tot starts at zero, so the merges below need no separate first-state case
-        uint32_t z[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) z[k] = 0u;
-#pragma unroll 1
-        for (int c0 = 0; c0 < DP; c0 += 16) tmem_st16(otot + c0, z);
-        tmem_wait_st();
-      }
+      // O_tot starts at zero, so the merges below need no separate first-state case
+#pragma unroll 4
+      for (int c = 0; c < DP; ++c) orow[c * 128] = 0.f;
       // (1) cached states of the REUSE pairs: merged first, while the MMA and
       //     softmax warps compute the item's first fresh state
       for (int j = 0; j < G.P; ++j) {
@@ -624,29 +630,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
         const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
-        for (int c1 = 0; c1 < DP; c1 += 64) {             // up to 64 cached columns in flight together
-          constexpr int kG = DP < 64 ? DP / 4 : 16;
-          float4 cv[kG];
+        for (int c1 = 0; c1 < D; c1 += 32) {             // 32 cached columns in flight together
+          float4 cv[8];
 #pragma unroll
-          for (int c = 0; c < kG; ++c)
-            cv[c] = (c1 + 4 * c < DP && valid && nonempty && c1 + 4 * c < D) ? __ldcs(src + c1 / 4 + c) : z4;
+          for (int c = 0; c < 8; ++c)
+            cv[c] = (c1 + 4 * c < D && valid && nonempty) ? __ldcs(src + c1 / 4 + c) : z4;
 #pragma unroll
-          for (int c0 = c1; c0 < DP && c0 < c1 + 64; c0 += 16) {
-            uint32_t ot[16];
-            tmem_ld16(otot + c0, ot);
-            tmem_wait_ld();
-#pragma unroll
-            for (int jj = 0; jj < 16; jj += 4) {
-              const float4 x = cv[(c0 - c1 + jj) / 4];
-              ot[jj + 0] = f2u(fmaf(a, u2f(ot[jj + 0]), b * x.x));
-              ot[jj + 1] = f2u(fmaf(a, u2f(ot[jj + 1]), b * x.y));
-              ot[jj + 2] = f2u(fmaf(a, u2f(ot[jj + 2]), b * x.z));
-              ot[jj + 3] = f2u(fmaf(a, u2f(ot[jj + 3]), b * x.w));
+          for (int c = 0; c < 8; ++c) {
+            if (c1 + 4 * c < D) {
+              float* o = orow + (c1 + 4 * c) * 128;
+              o[0] = fmaf(a, o[0], b * cv[c].x);
+              o[128] = fmaf(a, o[128], b * cv[c].y);
+              o[256] = fmaf(a, o[256], b * cv[c].z);
+              o[384] = fmaf(a, o[384], b * cv[c].w);
             }
-            tmem_st16(otot + c0, ot);
           }
         }
-        tmem_wait_st();
         if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
         have = have || nonempty;
       }
@@ -671,9 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[C::bStFree + st]);
         if (!warp_wait(&bars[C::bODSeg], cseg & 1, abort_flag, p.status, lim)) goto ep_done;
-
         tc_fence_after();
-        // O_part -> registers, then hand O_part straight back to the MMA warp
+        // O_part -> registers, then hand O_part straight back to the MMA warps
         uint32_t op[DP];
 #pragma unroll
         for (int c0 = 0; c0 < DP; c0 += 16) tmem_ld16p(opart + c0, op + c0);
@@ -696,71 +694,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const float inv_tot = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
         const float inv_new = l_new > 0.f ? 1.f / l_new : 0.f;
 #pragma unroll
-        for (int c0 = 0; c0 < DP; c0 += 16) {
-          uint32_t ot[16];
-          tmem_ld16(otot + c0, ot);
-          tmem_wait_ld();
+        for (int c = 0; c < D; c += 4) {
+          float old[4], nw[4], x[4];
 #pragma unroll
-          for (int jj = 0; jj < 16; jj += 4) {
-            float old[4], nw[4], x[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              old[k] = u2f(ot[jj + k]);
-              x[k] = u2f(op[c0 + jj + k]);
-              nw[k] = fmaf(a, old[k], b * x[k]);
-              ot[jj + k] = f2u(nw[k]);
-            }
-            if (valid && c0 + jj < D) {
-              if (!WIN) {
-                __stcs(reinterpret_cast<float4*>(p.cache_O + slot * D + c0 + jj),
-                       make_float4(x[0] * inv_l, x[1] * inv_l, x[2] * inv_l, x[3] * inv_l));
-              } else if (make_r) {
-                float4 v;
-                v.x = nw[0] * inv_new - old[0] * inv_tot;
-                v.y = nw[1] * inv_new - old[1] * inv_tot;
-                v.z = nw[2] * inv_new - old[2] * inv_tot;
-                v.w = nw[3] * inv_new - old[3] * inv_tot;
-                __stcs(reinterpret_cast<float4*>(p.R + ((size_t)h * G.S + qrow) * D + c0 + jj), v);
-              }
+          for (int k = 0; k < 4; ++k) {
+            old[k] = orow[(c + k) * 128];
+            x[k] = u2f(op[c + k]);
+            nw[k] = fmaf(a, old[k], b * x[k]);
+            orow[(c + k) * 128] = nw[k];
+          }
+          if (valid) {
+            if (!WIN) {
+              __stcs(reinterpret_cast<float4*>(p.cache_O + slot * D + c),
+                     make_float4(x[0] * inv_l, x[1] * inv_l, x[2] * inv_l, x[3] * inv_l));
+            } else if (make_r) {
+              float4 v;
+              v.x = nw[0] * inv_new - old[0] * inv_tot;
+              v.y = nw[1] * inv_new - old[1] * inv_tot;
+              v.z = nw[2] * inv_new - old[2] * inv_tot;
+              v.w = nw[3] * inv_new - old[3] * inv_tot;
+              __stcs(reinterpret_cast<float4*>(p.R + ((size_t)h * G.S + qrow) * D + c), v);
             }
           }
-          tmem_st16(otot + c0, ot);
         }
-        tmem_wait_st();
         if (!WIN && valid) __stcs(p.cache_L + slot, nonempty ? (m_s + lg2(l_s)) * kLn2 : kNegInf);
         if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
         have = have || nonempty;
         ++cseg;
       }
       // final: O = O_tot / l_tot (+ R), LSE = m_tot + log2(l_tot), in natural units
-      {
+      if (valid) {
         const float inv = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.O) + ((size_t)h * G.S + qrow) * D;
         const float* rr = p.R + ((size_t)h * G.S + qrow) * D;
-#pragma unroll 1
-        for (int c0 = 0; c0 < DP; c0 += 16) {
-          uint32_t ot[16];
-          tmem_ld16(otot + c0, ot);
-          tmem_wait_ld();
-          if (valid) {
-#pragma unroll
-            for (int j = 0; j < 16; j += 4) {
-              if (c0 + j < D) {
-                float v0 = u2f(ot[j]) * inv, v1 = u2f(ot[j + 1]) * inv;
-                float v2 = u2f(ot[j + 2]) * inv, v3 = u2f(ot[j + 3]) * inv;
-                if (use_r) {
-                  const float4 rv = __ldcs(reinterpret_cast<const float4*>(rr + c0 + j));
-                  v0 += rv.x; v1 += rv.y; v2 += rv.z; v3 += rv.w;
-                }
-                uint2 pk;
-                pk.x = pack_bf16x2(v0, v1);
-                pk.y = pack_bf16x2(v2, v3);
-                __stcs(reinterpret_cast<uint2*>(dst + c0 + j), pk);
-              }
-            }
+#pragma unroll 2
+        for (int c = 0; c < D; c += 4) {
+          float v0 = orow[c * 128] * inv, v1 = orow[(c + 1) * 128] * inv;
+          float v2 = orow[(c + 2) * 128] * inv, v3 = orow[(c + 3) * 128] * inv;
+          if (use_r) {
+            const float4 rv = __ldcs(reinterpret_cast<const float4*>(rr + c));
+            v0 += rv.x; v1 += rv.y; v2 += rv.z; v3 += rv.w;
           }
+          uint2 pk;
+          pk.x = pack_bf16x2(v0, v1);
+          pk.y = pack_bf16x2(v2, v3);
+          __stcs(reinterpret_cast<uint2*>(dst + c), pk);
         }
-        if (valid) __stcs(p.L + (size_t)h * G.S + qrow, (have && l_tot > 0.f) ? (m_tot + lg2(l_tot)) * kLn2 : kNegInf);
+        __stcs(p.L + (size_t)h * G.S + qrow, (have && l_tot > 0.f) ? (m_tot + lg2(l_tot)) * kLn2 : kNegInf);
       }
     }
   ep_done:

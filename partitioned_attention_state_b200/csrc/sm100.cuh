@@ -110,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, v
 // DT_ERR_TIMEOUT-style `code` in *status (first error wins).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int32_t* status, int32_t code, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test(bar, parity)) return true;      // non-blocking check first: most waits find the phase done
   return mbar_wait_slow(bar, parity, abort, status, code, limit_ns);
 }
 
