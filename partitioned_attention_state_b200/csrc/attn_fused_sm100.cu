@@ -94,7 +94,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when t
 __constant__ uint64_t* g_dt_trace = nullptr;   // constant bank: no global load per stamp
 #define DT_TR(ev, idx)                                                                             \
   do {                                                                                             \
-    if (blockIdx.x == 0 && (threadIdx.x & 31) == 0 && g_dt_trace && (idx) < 4096)                 \
+    if (blockIdx.x == 0 && g_dt_trace && (idx) < 4096)   /* all lanes: no divergence */          \
       g_dt_trace[(ev) * 4096 + (idx)] = clock64();                                                 \
   } while (0)
 #else
@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         if (nt == 0) continue;
         // running max (log2 units) and partial row sums of rows ra, rb
         float ma = kNegInf, mb = kNegInf;
-        float la[4] = {0.f, 0.f, 0.f, 0.f}, lb[4] = {0.f, 0.f, 0.f, 0.f};
+        uint64_t la[2] = {0ull, 0ull}, lb[2] = {0ull, 0ull};      // packed pairs of partial sums
         const bool precise = WIN && seg == 0;
         for (int i = 0; i < nt; ++i, ++g) {
           const uint32_t sb = g % C::kNS;
@@ -517,11 +517,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               tmem_st_16x256b_x2(oc + c0, o);
             }
             tmem_wait_st();
+            const uint64_t aa = pk2(alpha_a, alpha_a), ab = pk2(alpha_b, alpha_b);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) { la[k] *= alpha_a; lb[k] *= alpha_b; }
+            for (int k = 0; k < 2; ++k) { la[k] = fma2(la[k], aa, 0ull); lb[k] = fma2(lb[k], ab, 0ull); }
           }
           ma = na; mb = nb;
           const float mra = (ma == kNegInf) ? 0.f : ma, mrb = (mb == kNegInf) ? 0.f : mb;
+          const uint64_t sl2x2 = pk2(sl2, sl2), nma = pk2(-mra, -mra), nmb = pk2(-mrb, -mrb);
           // exponentials, 8 repetitions (32 P columns) per TMEM store
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
@@ -529,13 +531,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 #pragma unroll
             for (int r4 = 0; r4 < 8; ++r4) {
               const int e = 4 * (8 * hf + r4);
-              const float x0 = fmaf(u2f(sr[e]), sl2, -mra), x1 = fmaf(u2f(sr[e + 1]), sl2, -mra);
-              const float x2 = fmaf(u2f(sr[e + 2]), sl2, -mrb), x3 = fmaf(u2f(sr[e + 3]), sl2, -mrb);
+              float x0, x1, x2, x3;
+              upk2(fma2(pk2(u2f(sr[e]), u2f(sr[e + 1])), sl2x2, nma), x0, x1);
+              upk2(fma2(pk2(u2f(sr[e + 2]), u2f(sr[e + 3])), sl2x2, nmb), x2, x3);
               const bool emu = kEmuMod > 0 && !masked && !precise && (r4 % (kEmuMod > 0 ? kEmuMod : 1)) == kEmuMod - 1;
               const float p0 = emu ? dt_exp2_fma(x0) : ex2(x0), p1 = emu ? dt_exp2_fma(x1) : ex2(x1);
               const float p2 = emu ? dt_exp2_fma(x2) : ex2(x2), p3 = emu ? dt_exp2_fma(x3) : ex2(x3);
-              la[r4 & 3] += p0 + p1;
-              lb[r4 & 3] += p2 + p3;
+              la[r4 & 1] = add2(la[r4 & 1], pk2(p0, p1));
+              lb[r4 & 1] = add2(lb[r4 & 1], pk2(p2, p3));
               ph[2 * r4] = pack_bf16x2(p0, p1);
               ph[2 * r4 + 1] = pack_bf16x2(p2, p3);
               if (precise) {                      // bf16 residuals overwrite the consumed logits
@@ -562,7 +565,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           if (warp == 7) DT_TR(13, g);
         }
         {
-          float sa = ((la[0] + la[1]) + (la[2] + la[3])), sbm = ((lb[0] + lb[1]) + (lb[2] + lb[3]));
+          float sa, sbm;
+          {
+            float u0, u1, v0, v1;
+            upk2(add2(la[0], la[1]), u0, u1);
+            upk2(add2(lb[0], lb[1]), v0, v1);
+            sa = u0 + u1;
+            sbm = v0 + v1;
+          }
           sa += __shfl_xor_sync(0xffffffffu, sa, 1);
           sbm += __shfl_xor_sync(0xffffffffu, sbm, 1);
           sa += __shfl_xor_sync(0xffffffffu, sa, 2);
