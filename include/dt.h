@@ -131,7 +131,9 @@ DT_API int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, 
  *               [2] fresh states written and [3] cached states read, each
  *               counted per (query tile, key set, head)
  *   d_status    int32 device status word (see conventions)
- * The host validates shapes and alignment before any launch.  One launch. */
+ * The host validates shapes and alignment before any launch.  One launch.
+ * Partition mode supports at most 64 partitions (DT_ERR_UNSUPPORTED above);
+ * d_plan must be 16-byte aligned like every other pointer. */
 DT_API int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan,
                           const void* Q, const void* K, const void* V,
                           float* cache_O, float* cache_L, float* R,

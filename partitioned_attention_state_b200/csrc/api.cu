@@ -82,10 +82,11 @@ extern "C" int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_p
   if (!shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (win ? p->window < 1 : p->P < 1) return DT_ERR_INVALID;
   if (p->D != 64 && p->D != 72 && p->D != 128) return DT_ERR_UNSUPPORTED;
+  if (!win && p->P > 64) return DT_ERR_UNSUPPORTED;      // the kernel keeps a plan row as a 64-bit mask
   if (p->H == 0 || p->S == 0) return DT_OK;
   if (!d_plan || !Q || !K || !V || !O || !L || !d_status) return DT_ERR_INVALID;
   if (win ? !R : (!cache_O || !cache_L)) return DT_ERR_INVALID;
-  const void* ptrs[] = {Q, K, V, O, L, d_status};
+  const void* ptrs[] = {d_plan, Q, K, V, O, L, d_status};
   for (const void* q : ptrs)
     if (!aligned16(q)) return DT_ERR_UNSUPPORTED;
   if ((cache_O && !aligned16(cache_O)) || (cache_L && !aligned16(cache_L)) || (R && !aligned16(R)) ||

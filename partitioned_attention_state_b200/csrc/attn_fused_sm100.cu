@@ -140,10 +140,30 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
+// Plan row of a query tile as a bit mask (bit s set: key set s is COMPUTE).
+// Read once per item with independent loads; the plan stays in global
+// memory, and testing it byte by byte at every key-set step put a chain of
+// dependent loads between consecutive key sets.  At most 64 key sets.
+__device__ __forceinline__ uint64_t plan_mask(const uint8_t* prow, int P) {
+  uint64_t m = 0;
+  if ((P & 3) == 0) {                       // rows start 4-byte aligned
+#pragma unroll 4
+    for (int s = 0; s < P; s += 4) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(prow + s);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) m |= (uint64_t)(((w >> (8 * b)) & 0xffu) == DT_PLAN_COMPUTE) << (s + b);
+    }
+  } else {
+    for (int s = 0; s < P; ++s) m |= (uint64_t)(prow[s] == DT_PLAN_COMPUTE) << s;
+  }
+  return m;
+}
+__device__ __forceinline__ bool is_compute(uint64_t cm, int seg) { return (cm >> seg) & 1u; }
+
 template <bool WIN>
-__device__ __forceinline__ bool item_has_compute(const Geom& G, int qt, const uint8_t* prow) {
+__device__ __forceinline__ bool item_has_compute(const Geom& G, int qt, uint64_t cm) {
   for (int s = 0; s < G.P; ++s)
-    if (prow[s] == DT_PLAN_COMPUTE && key_set<WIN>(G, qt, s).ntiles() > 0) return true;
+    if (is_compute(cm, s) && key_set<WIN>(G, qt, s).ntiles() > 0) return true;
   return false;
 }
 
@@ -230,11 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   if (warp == kWarpTmaK && lane == 0) {
     for (int i = 0; i < C::kNumBars; ++i) mbar_init(&bars[i], 1);
     for (int i = 0; i < C::kNS; ++i) mbar_init(&bars[C::bPFull + i], 8 * 32);   // every softmax thread arrives
+    // every thread of the arriving role arrives (no single-lane branches)
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[C::bStFull + i], 8);
-      mbar_init(&bars[C::bStFree + i], 4);    // one arrival per epilogue warp
+      mbar_init(&bars[C::bStFull + i], 8 * 32);
+      mbar_init(&bars[C::bStFree + i], 4 * 32);
     }
-    mbar_init(&bars[C::bOFree], 4);
+    mbar_init(&bars[C::bOFree], 4 * 32);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async();
@@ -270,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       uint32_t g = 0, nq = 0;
       for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
         const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
-        const uint8_t* prow = p.plan + (size_t)qt * G.P;
-        if (!item_has_compute<WIN>(G, qt, prow)) continue;
+        const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+        if (!item_has_compute<WIN>(G, qt, cm)) continue;
         if (is_k) {
           const QTile t = query_tile<WIN>(G, qt);
           if (nq > 0 && !mbar_wait(&bars[C::bQEmpty], (nq - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
@@ -285,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         }
         for (int j = 0; j < G.P; ++j) {
           const int seg = visit_seg<WIN>(G, idx, j);
-          if (prow[seg] != DT_PLAN_COMPUTE) continue;
+          if (!is_compute(cm, seg)) continue;
           const KeySet ks = key_set<WIN>(G, qt, seg);
           const int nt = ks.ntiles();
           for (int i = 0; i < nt; ++i, ++g) {
@@ -326,14 +347,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
-        const uint8_t* prow = p.plan + (size_t)qt * G.P;
-        if (!item_has_compute<WIN>(G, qt, prow)) continue;
+        const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+        if (!item_has_compute<WIN>(G, qt, cm)) continue;
         if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
         ++nq;
         tc_fence_after();
         for (int j = 0; j < G.P && ok; ++j) {
           const int seg = visit_seg<WIN>(G, idx, j);
-          if (prow[seg] != DT_PLAN_COMPUTE) continue;
+          if (!is_compute(cm, seg)) continue;
           const int nt = key_set<WIN>(G, qt, seg).ntiles();
           if (nt == 0) continue;
           for (int i = 0; i < nt; ++i, ++g) {
@@ -397,11 +418,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       bool ok = true;
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
-        const uint8_t* prow = p.plan + (size_t)qt * G.P;
-        if (!item_has_compute<WIN>(G, qt, prow)) continue;
+        const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+        if (!item_has_compute<WIN>(G, qt, cm)) continue;
         for (int j = 0; j < G.P && ok; ++j) {
           const int seg = visit_seg<WIN>(G, idx, j);
-          if (prow[seg] != DT_PLAN_COMPUTE) continue;
+          if (!is_compute(cm, seg)) continue;
           const int nt = key_set<WIN>(G, qt, seg).ntiles();
           if (nt == 0) continue;
           for (int i = 0; i < nt && ok; ++i, ++g)
@@ -431,14 +452,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     uint32_t g = 0, cseg = 0;
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const int qt = idx - (idx / G.nqt) * G.nqt;
-      const uint8_t* prow = p.plan + (size_t)qt * G.P;
-      if (!item_has_compute<WIN>(G, qt, prow)) continue;
+      const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+      if (!item_has_compute<WIN>(G, qt, cm)) continue;
       const QTile t = query_tile<WIN>(G, qt);
       const int qa = t.q0 + ra, qb = t.q0 + rb;
       const int q1 = t.q0 + t.rows - 1;
       for (int j = 0; j < G.P; ++j) {
         const int seg = visit_seg<WIN>(G, idx, j);
-        if (prow[seg] != DT_PLAN_COMPUTE) continue;
+        if (!is_compute(cm, seg)) continue;
         const KeySet ks = key_set<WIN>(G, qt, seg);
         const int nt = ks.ntiles();
         if (nt == 0) continue;
@@ -580,14 +601,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           const uint32_t st = cseg & 1;
           if (cseg >= 2 && !warp_wait(&bars[C::bStFree + st], ((cseg >> 1) - 1) & 1, abort_flag, p.status, lim))
             goto sm_done;
-          if ((lane & 3) == 0) {
-            stat_m[st * 128 + ra] = ma;
-            stat_l[st * 128 + ra] = sa;
-            stat_m[st * 128 + rb] = mb;
-            stat_l[st * 128 + rb] = sbm;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[C::bStFull + st]);
+          // the 4 threads of a row hold the same values: all of them write
+          stat_m[st * 128 + ra] = ma;
+          stat_l[st * 128 + ra] = sa;
+          stat_m[st * 128 + rb] = mb;
+          stat_l[st * 128 + rb] = sbm;
+          mbar_arrive(&bars[C::bStFull + st]);
           ++cseg;
         }
       }
@@ -609,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     uint32_t n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
-      const uint8_t* prow = p.plan + (size_t)qt * G.P;
+      const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
       const QTile t = query_tile<WIN>(G, qt);
       const int qrow = t.q0 + r;
       const bool valid = r < t.rows;
@@ -618,54 +637,63 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       // O_tot starts at zero, so the merges below need no separate first-state case
 #pragma unroll 4
       for (int c = 0; c < DP; ++c) orow[c * 128] = 0.f;
-      // (1) cached states of the REUSE pairs: merged first, while the MMA and
-      //     softmax warps compute the item's first fresh state
-      for (int j = 0; j < G.P; ++j) {
-        const int seg = visit_seg<WIN>(G, idx, j);
-        if (prow[seg] == DT_PLAN_COMPUTE) continue;
-        if (r == 0) { n_skip += counted_blocks<WIN>(G, qt, seg); ++n_read; }
-        if (WIN) { use_r = true; continue; }     // complement reused: add R at the end
-        const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
-        const float lse_c = valid ? __ldcs(p.cache_L + slot) : kNegInf;
-        const bool nonempty = lse_c > kNegInf;
-        const float m_c = lse_c * kLog2e;
-        float a, b, m_new;
-        if (!have) { m_new = m_c; a = 0.f; b = nonempty ? 1.f : 0.f; }
-        else {
-          m_new = nonempty ? fmaxf(m_tot, m_c) : m_tot;
-          a = ex2(m_tot - m_new);
-          b = nonempty ? ex2(m_c - m_new) : 0.f;
-        }
-        const float l_new = a * l_tot + b;
-        const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
-        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      // Cached states of the REUSE pairs are composed into O_tot while the
+      // next fresh state is not ready yet (and the rest after the last one):
+      // their loads are latency-bound, and reading O_part promptly is what the
+      // MMA warps wait on.  jr walks the key sets in visiting order.
+      int jr = 0;
+      auto merge_next_reused = [&]() {
+        for (; jr < G.P; ++jr) {
+          const int seg = visit_seg<WIN>(G, idx, jr);
+          if (is_compute(cm, seg)) continue;
+          n_skip += counted_blocks<WIN>(G, qt, seg);   // same in every lane; thread 0 reports
+          ++n_read;
+          if (WIN) { use_r = true; continue; }     // complement reused: add R at the end
+          const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
+          const float lse_c = valid ? __ldcs(p.cache_L + slot) : kNegInf;
+          const bool nonempty = lse_c > kNegInf;
+          const float m_c = lse_c * kLog2e;
+          float a, b, m_new;
+          if (!have) { m_new = m_c; a = 0.f; b = nonempty ? 1.f : 0.f; }
+          else {
+            m_new = nonempty ? fmaxf(m_tot, m_c) : m_tot;
+            a = ex2(m_tot - m_new);
+            b = nonempty ? ex2(m_c - m_new) : 0.f;
+          }
+          const float l_new = a * l_tot + b;
+          const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
+          const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
-        for (int c1 = 0; c1 < D; c1 += 32) {             // 32 cached columns in flight together
-          float4 cv[8];
+          for (int c1 = 0; c1 < D; c1 += 32) {             // 32 cached columns in flight together
+            float4 cv[8];
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            cv[c] = (c1 + 4 * c < D && valid && nonempty) ? __ldcs(src + c1 / 4 + c) : z4;
+            for (int c = 0; c < 8; ++c)
+              cv[c] = (c1 + 4 * c < D && valid && nonempty) ? __ldcs(src + c1 / 4 + c) : z4;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            if (c1 + 4 * c < D) {
-              float* o = orow + (c1 + 4 * c) * 128;
-              o[0] = fmaf(a, o[0], b * cv[c].x);
-              o[128] = fmaf(a, o[128], b * cv[c].y);
-              o[256] = fmaf(a, o[256], b * cv[c].z);
-              o[384] = fmaf(a, o[384], b * cv[c].w);
+            for (int c = 0; c < 8; ++c) {
+              if (c1 + 4 * c < D) {
+                float* o = orow + (c1 + 4 * c) * 128;
+                o[0] = fmaf(a, o[0], b * cv[c].x);
+                o[128] = fmaf(a, o[128], b * cv[c].y);
+                o[256] = fmaf(a, o[256], b * cv[c].z);
+                o[384] = fmaf(a, o[384], b * cv[c].w);
+              }
             }
           }
+          if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
+          have = have || nonempty;
+          ++jr;
+          return;
         }
-        if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
-        have = have || nonempty;
-      }
+      };
       // (2) fresh states, in the order the MMA produces them
       for (int j = 0; j < G.P; ++j) {
         const int seg = visit_seg<WIN>(G, idx, j);
-        if (prow[seg] != DT_PLAN_COMPUTE) continue;
+        if (!is_compute(cm, seg)) continue;
         const int nt = key_set<WIN>(G, qt, seg).ntiles();
         const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
-        if (r == 0) { n_comp += counted_blocks<WIN>(G, qt, seg); ++n_fresh; }
+        n_comp += counted_blocks<WIN>(G, qt, seg);
+        ++n_fresh;
         if (nt == 0) {             // empty key set: the identity state
           if (!WIN && valid) {
             float4* dst = reinterpret_cast<float4*>(p.cache_O + slot * D);
@@ -675,10 +703,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           continue;
         }
         const uint32_t st = cseg & 1;
+        while (jr < G.P && !__shfl_sync(0xffffffffu, (int)mbar_test(&bars[C::bODSeg], cseg & 1), 0))
+          merge_next_reused();
         if (!warp_wait(&bars[C::bStFull + st], (cseg >> 1) & 1, abort_flag, p.status, lim)) goto ep_done;
         const float m_s = stat_m[st * 128 + r], l_s = stat_l[st * 128 + r];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[C::bStFree + st]);
+        mbar_arrive(&bars[C::bStFree + st]);
         if (!warp_wait(&bars[C::bODSeg], cseg & 1, abort_flag, p.status, lim)) goto ep_done;
         tc_fence_after();
         // O_part -> registers, then hand O_part straight back to the MMA warps
@@ -687,8 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         for (int c0 = 0; c0 < DP; c0 += 16) tmem_ld16p(opart + c0, op + c0);
         tmem_wait_ld();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[C::bOFree]);
+        mbar_arrive(&bars[C::bOFree]);
         if (warp == kWarpEpi) DT_TR(7, cseg);
         const bool nonempty = l_s > 0.f;
         const float inv_l = nonempty ? 1.f / l_s : 0.f;
@@ -732,6 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         have = have || nonempty;
         ++cseg;
       }
+      while (jr < G.P) merge_next_reused();
       // final: O = O_tot / l_tot (+ R), LSE = m_tot + log2(l_tot), in natural units
       if (valid) {
         const float inv = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
