@@ -144,15 +144,18 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // Read once per item with independent loads; the plan stays in global
 // memory, and testing it byte by byte at every key-set step put a chain of
 // dependent loads between consecutive key sets.  At most 64 key sets.
+__device__ __forceinline__ uint32_t mask4(uint32_t w) {     // 4 plan bytes (0/1) -> 4 bits
+  w &= 0x01010101u;
+  return (w | (w >> 7) | (w >> 14) | (w >> 21)) & 0xfu;
+}
+template <bool WIN>
 __device__ __forceinline__ uint64_t plan_mask(const uint8_t* prow, int P) {
   uint64_t m = 0;
-  if ((P & 3) == 0) {                       // rows start 4-byte aligned
+  if (WIN) {                                // two key sets
+    m = (uint64_t)(prow[0] == DT_PLAN_COMPUTE) | ((uint64_t)(prow[1] == DT_PLAN_COMPUTE) << 1);
+  } else if ((P & 3) == 0) {                // rows start 4-byte aligned
 #pragma unroll 4
-    for (int s = 0; s < P; s += 4) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(prow + s);
-#pragma unroll
-      for (int b = 0; b < 4; ++b) m |= (uint64_t)(((w >> (8 * b)) & 0xffu) == DT_PLAN_COMPUTE) << (s + b);
-    }
+    for (int s = 0; s < P; s += 4) m |= (uint64_t)mask4(*reinterpret_cast<const uint32_t*>(prow + s)) << s;
   } else {
     for (int s = 0; s < P; ++s) m |= (uint64_t)(prow[s] == DT_PLAN_COMPUTE) << s;
   }
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       uint32_t g = 0, nq = 0;
       for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
         const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
-        const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+        const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         if (!item_has_compute<WIN>(G, qt, cm)) continue;
         if (is_k) {
           const QTile t = query_tile<WIN>(G, qt);
@@ -347,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
-        const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+        const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         if (!item_has_compute<WIN>(G, qt, cm)) continue;
         if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
         ++nq;
@@ -418,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       bool ok = true;
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
-        const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+        const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         if (!item_has_compute<WIN>(G, qt, cm)) continue;
         for (int j = 0; j < G.P && ok; ++j) {
           const int seg = visit_seg<WIN>(G, idx, j);
@@ -452,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     uint32_t g = 0, cseg = 0;
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const int qt = idx - (idx / G.nqt) * G.nqt;
-      const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+      const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
       if (!item_has_compute<WIN>(G, qt, cm)) continue;
       const QTile t = query_tile<WIN>(G, qt);
       const int qa = t.q0 + ra, qb = t.q0 + rb;
@@ -628,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     uint32_t n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
-      const uint64_t cm = plan_mask(p.plan + (size_t)qt * G.P, G.P);
+      const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
       const QTile t = query_tile<WIN>(G, qt);
       const int qrow = t.q0 + r;
       const bool valid = r < t.rows;
