@@ -175,13 +175,16 @@ __device__ __forceinline__ bool item_has_compute(const Geom& G, int qt, uint64_t
 // free, so any order gives the same result; rotating the start per item keeps
 // the CTAs that run together from streaming the same K/V tile at once.
 template <bool WIN>
-__device__ __forceinline__ int visit_seg(const Geom& G, int idx, int j) {
-  if (WIN) return j;                 // window set before its complement
-  int s = j + idx % G.P;
+__device__ __forceinline__ int seg_rotation(const Geom& G, int idx) { return WIN ? 0 : idx % G.P; }
+template <bool WIN>
+__device__ __forceinline__ int visit_seg(const Geom& G, int rot, int j) {
+  if (WIN) return j;                          // window set before its complement
+  const int s = j + rot;
   return s >= G.P ? s - G.P : s;
 }
-__device__ __forceinline__ int visit_tile(const KeySet& ks, int nt, int idx, int seg, int i) {
-  int k = i + (idx * 5 + seg * 3) % nt;
+__device__ __forceinline__ int tile_rotation(int nt, int idx, int seg) { return (idx * 5 + seg * 3) % nt; }
+__device__ __forceinline__ int visit_tile(const KeySet& ks, int nt, int off, int i) {
+  const int k = i + off;
   return ks.tile(k >= nt ? k - nt : k);
 }
 
@@ -295,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
         const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
+        const int rot = seg_rotation<WIN>(G, idx);
         if (!item_has_compute<WIN>(G, qt, cm)) continue;
         if (is_k) {
           const QTile t = query_tile<WIN>(G, qt);
@@ -308,16 +312,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           ++nq;
         }
         for (int j = 0; j < G.P; ++j) {
-          const int seg = visit_seg<WIN>(G, idx, j);
+          const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
           const KeySet ks = key_set<WIN>(G, qt, seg);
           const int nt = ks.ntiles();
+          const int toff = nt > 0 ? tile_rotation(nt, idx, seg) : 0;
           for (int i = 0; i < nt; ++i, ++g) {
             const int st = g % C::kStages;
             if (g >= (uint32_t)C::kStages &&
                 !mbar_wait(&empty[st], ((g / C::kStages) - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
               goto tma_done;
-            const int row0 = ks.base + visit_tile(ks, nt, idx, seg, i) * kTile;
+            const int row0 = ks.base + visit_tile(ks, nt, toff, i) * kTile;
             uint8_t* dst = ring + st * C::kTileBytes;
             DT_TR(is_k ? 8 : 9, g);
             mbar_arrive_expect_tx(&full[st], C::kTileBytes);
@@ -351,12 +356,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
+        const int rot = seg_rotation<WIN>(G, idx);
         if (!item_has_compute<WIN>(G, qt, cm)) continue;
         if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
         ++nq;
         tc_fence_after();
         for (int j = 0; j < G.P && ok; ++j) {
-          const int seg = visit_seg<WIN>(G, idx, j);
+          const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
           const int nt = key_set<WIN>(G, qt, seg).ntiles();
           if (nt == 0) continue;
@@ -422,9 +428,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
+        const int rot = seg_rotation<WIN>(G, idx);
         if (!item_has_compute<WIN>(G, qt, cm)) continue;
         for (int j = 0; j < G.P && ok; ++j) {
-          const int seg = visit_seg<WIN>(G, idx, j);
+          const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
           const int nt = key_set<WIN>(G, qt, seg).ntiles();
           if (nt == 0) continue;
@@ -456,16 +463,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const int qt = idx - (idx / G.nqt) * G.nqt;
       const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
+      const int rot = seg_rotation<WIN>(G, idx);
       if (!item_has_compute<WIN>(G, qt, cm)) continue;
       const QTile t = query_tile<WIN>(G, qt);
       const int qa = t.q0 + ra, qb = t.q0 + rb;
       const int q1 = t.q0 + t.rows - 1;
       for (int j = 0; j < G.P; ++j) {
-        const int seg = visit_seg<WIN>(G, idx, j);
+        const int seg = visit_seg<WIN>(G, rot, j);
         if (!is_compute(cm, seg)) continue;
         const KeySet ks = key_set<WIN>(G, qt, seg);
         const int nt = ks.ntiles();
         if (nt == 0) continue;
+        const int toff = tile_rotation(nt, idx, seg);
         // running max (log2 units) and partial row sums of rows ra, rb
         float ma = kNegInf, mb = kNegInf;
         uint64_t la[2] = {0ull, 0ull}, lb[2] = {0ull, 0ull};      // packed pairs of partial sums
@@ -477,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           if (warp == 0) DT_TR(2, g);
           if (warp == 7) DT_TR(14, g);
           tc_fence_after();
-          const int tile = visit_tile(ks, nt, idx, seg, i);
+          const int tile = visit_tile(ks, nt, toff, i);
           const int k0 = ks.base + tile * kTile;
           const int kvalid = imin(kTile, ks.kend - k0);
           const uint32_t sc = tmem + lane_base + C::kColS + sb * 128;
@@ -632,6 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
       const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
+      const int rot = seg_rotation<WIN>(G, idx);
       const QTile t = query_tile<WIN>(G, qt);
       const int qrow = t.q0 + r;
       const bool valid = r < t.rows;
@@ -647,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       int jr = 0;
       auto merge_next_reused = [&]() {
         for (; jr < G.P; ++jr) {
-          const int seg = visit_seg<WIN>(G, idx, jr);
+          const int seg = visit_seg<WIN>(G, rot, jr);
           if (is_compute(cm, seg)) continue;
           n_skip += counted_blocks<WIN>(G, qt, seg);   // same in every lane; thread 0 reports
           ++n_read;
@@ -691,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       };
       // (2) fresh states, in the order the MMA produces them
       for (int j = 0; j < G.P; ++j) {
-        const int seg = visit_seg<WIN>(G, idx, j);
+        const int seg = visit_seg<WIN>(G, rot, j);
         if (!is_compute(cm, seg)) continue;
         const int nt = key_set<WIN>(G, qt, seg).ntiles();
         const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
