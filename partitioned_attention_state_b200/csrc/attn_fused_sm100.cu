@@ -130,6 +130,20 @@ struct Cfg {
 constexpr int kEmuMod = 0;
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+// A softmax thread holds columns c_j = 8*(j/2) + cq + (j%2), j = 0..31, of
+// its rows (increasing in j).  cols_below(x): how many of them are < x;
+// cols_in(lo, hi): bit j set iff lo <= c_j <= hi.
+__device__ __forceinline__ int cols_below(int x, int cq) {
+  const int y = x - cq;
+  return imin(imax((y + 7) >> 3, 0), 16) + imin(imax((y + 6) >> 3, 0), 16);
+}
+__device__ __forceinline__ uint32_t cols_in(int lo, int hi, int cq) {
+  const int a = cols_below(lo, cq), b = cols_below(hi + 1, cq);
+  const uint32_t upto_b = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+  const uint32_t upto_a = a >= 32 ? 0xffffffffu : ((1u << a) - 1u);
+  return upto_b & ~upto_a;
+}
 __device__ __forceinline__ uint32_t f2u(float f) { return __float_as_uint(f); }
 
 // Warp-level wait: every lane checks the barrier itself (uniform control
@@ -501,16 +515,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
                                  : (wtile_touches(G, t.q0, q1, tile) ? 2 : 0);
           const bool masked = kvalid < kTile || mask_kind != 0;
           if (masked) {
+            // kept columns of rows ra and rb as bit masks over this thread's
+            // 32 columns (the band |i-j| <= hw is a column interval per row),
+            // then one bit test per element: compact code for the edge tiles
+            const uint32_t all = cols_in(0, kvalid - 1, cq);
+            uint32_t ka = all, kb = all;
+            if (mask_kind != 0) {
+              const uint32_t wa = cols_in(qa - G.hw - k0, qa + G.hw - k0, cq);
+              const uint32_t wb = cols_in(qb - G.hw - k0, qb + G.hw - k0, cq);
+              ka = mask_kind == 1 ? (all & wa) : (all & ~wa);
+              kb = mask_kind == 1 ? (all & wb) : (all & ~wb);
+            }
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
-              const int c = 8 * (e >> 2) + cq + (e & 1);
-              const int key = k0 + c;
-              const int q = (e & 2) ? qb : qa;
-              const int dist = q > key ? q - key : key - q;
-              bool keep = c < kvalid;
-              if (mask_kind == 1) keep = keep && dist <= G.hw;
-              if (mask_kind == 2) keep = keep && dist > G.hw;
-              if (!keep) sr[e] = f2u(kNegInf);
+              const uint32_t km = (e & 2) ? kb : ka;
+              if (!(km & (1u << (2 * (e >> 2) + (e & 1))))) sr[e] = f2u(kNegInf);
             }
           }
           // row maxima: two chains per row, then across the 4 threads of a row
@@ -532,7 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           const float mxa2 = mxa * sl2, mxb2 = mxb * sl2;
           const float na = (i == 0) ? mxa2 : ((mxa2 > ma + kRescaleThreshold) ? mxa2 : ma);
           const float nb = (i == 0) ? mxb2 : ((mxb2 > mb + kRescaleThreshold) ? mxb2 : mb);
-          const bool resa = (i > 0) && (na != ma), resb = (i > 0) && (nb != mb);
+          // a row that has seen only masked keys (max -inf) has O_part = 0 and
+          // l = 0: it takes the new reference without a rescale (and without
+          // waiting for the previous PV)
+          const bool resa = (i > 0) && (na != ma) && (ma != kNegInf);
+          const bool resb = (i > 0) && (nb != mb) && (mb != kNegInf);
           if (__any_sync(0xffffffffu, resa || resb)) {
             // O_part holds the previous tiles' sum: wait for its last PV, then rescale
             if (!warp_wait(&bars[C::bPVDone + (g - 1) % C::kNS], ((g - 1) / C::kNS) & 1, abort_flag, p.status, lim))
