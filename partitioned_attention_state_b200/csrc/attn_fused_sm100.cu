@@ -673,18 +673,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       // O_tot starts at zero, so the merges below need no separate first-state case
 #pragma unroll 4
       for (int c = 0; c < DP; ++c) orow[c * 128] = 0.f;
-      // Cached states of the REUSE pairs are composed into O_tot while the
-      // next fresh state is not ready yet (and the rest after the last one):
-      // their loads are latency-bound, and reading O_part promptly is what the
-      // MMA warps wait on.  jr walks the key sets in visiting order.
-      int jr = 0;
+      // Cached states of the REUSE pairs are composed into O_tot interleaved
+      // with the fresh ones, a fixed share before each fresh state (their
+      // loads are latency-bound; composing them all first would hold up the
+      // release of O_part that the MMA warps wait on).  The order depends
+      // only on the plan, so results are reproducible run to run.  jr walks
+      // the key sets in visiting order; merged counts reused sets done.
+      const int sets_fresh = __popcll(cm), sets_reused = G.P - sets_fresh;
+      int jr = 0, merged = 0, fi = 0;
       auto merge_next_reused = [&]() {
         for (; jr < G.P; ++jr) {
           const int seg = visit_seg<WIN>(G, rot, jr);
           if (is_compute(cm, seg)) continue;
           n_skip += counted_blocks<WIN>(G, qt, seg);   // same in every lane; thread 0 reports
           ++n_read;
-          if (WIN) { use_r = true; continue; }     // complement reused: add R at the end
+          if (WIN) { use_r = true; ++merged; continue; }   // complement reused: add R at the end
           const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
           const float lse_c = valid ? __ldcs(p.cache_L + slot) : kNegInf;
           const bool nonempty = lse_c > kNegInf;
@@ -719,6 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
           have = have || nonempty;
           ++jr;
+          ++merged;
           return;
         }
       };
@@ -739,8 +743,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           continue;
         }
         const uint32_t st = cseg & 1;
-        while (jr < G.P && !__shfl_sync(0xffffffffu, (int)mbar_test(&bars[C::bODSeg], cseg & 1), 0))
-          merge_next_reused();
+        ++fi;
+        while (jr < G.P && merged * sets_fresh < fi * sets_reused) merge_next_reused();
         if (!warp_wait(&bars[C::bStFull + st], (cseg >> 1) & 1, abort_flag, p.status, lim)) goto ep_done;
         const float m_s = stat_m[st * 128 + r], l_s = stat_l[st * 128 + r];
         mbar_arrive(&bars[C::bStFree + st]);

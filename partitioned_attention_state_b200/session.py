@@ -102,9 +102,44 @@ class Session:
         dt_attn_partial_fused(p, self.d_plan, self.Q, self.K, self.V, self.cache_O, self.cache_L, self.R, self.O,
                               self.L, self.counters, self.status, stream)
 
+    def capture_step(self, step: int, mode: Optional[int] = None,
+                     explicit: Optional[np.ndarray] = None) -> "StepGraph":
+        """Build the plan of `step` once and capture its fused launch in a CUDA
+        graph.  Replaying the graph repeats the step on the current contents of
+        the session's buffers with no host work (plan build, upload, launch
+        set-up), which is what small workloads are bound by.  The plan lives in
+        its own device buffer, so eager steps in between do not disturb it;
+        replays do not advance the host stamps."""
+        p, plan, counts = self.plan(step, mode, explicit)
+        gplan = torch.zeros_like(self.d_plan)
+        if self.nqt > 0:
+            gplan[: self.nqt].copy_(torch.from_numpy(np.ascontiguousarray(plan)))
+        # one eager launch first: per-process set-up (kernel attributes) stays out of the capture
+        dt_attn_partial_fused(p, gplan, self.Q, self.K, self.V, self.cache_O, self.cache_L, self.R, self.O, self.L,
+                              self.counters, self.status, torch.cuda.current_stream(self.device))
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            dt_attn_partial_fused(p, gplan, self.Q, self.K, self.V, self.cache_O, self.cache_L, self.R, self.O,
+                                  self.L, self.counters, self.status, side)
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        return StepGraph(graph, gplan, counts, plan)
+
     def check(self) -> None:
         """Synchronise and raise if a kernel reported a device-side error."""
         torch.cuda.synchronize(self.device)
         st = int(self.status[0].item())
         if st != 0:
             raise DtError(st, "device status")
+
+
+class StepGraph:
+    """A captured fused launch (see Session.capture_step)."""
+
+    def __init__(self, graph, d_plan, counts, plan):
+        self.graph, self.d_plan, self.counts, self.plan = graph, d_plan, counts, plan
+
+    def replay(self) -> dict:
+        self.graph.replay()
+        return self.counts
