@@ -148,8 +148,15 @@ def test_device_entry_points_validate_before_any_cuda_call():
     assert lib.dt_window_residual(0, 1, 8, 64, None, None, None, None, None, None) == dt.DT_ERR_INVALID
     pw = dt.params(1, 64, 64, 1, dt.DT_MODE_WINDOW, 0, 8, 1)
     assert lib.dt_state_cache_update(ctypes.byref(pw), *([None] * 7)) == dt.DT_ERR_INVALID
-    # misaligned device pointer is refused on the host
+    # the fused kernel keeps a plan row as a 64-bit mask: at most 64 partitions
+    p64 = dt.params(1, 128 * 65, 64, 65, dt.DT_MODE_ALL_COMPUTE, 0, 0, 1)
+    assert lib.dt_attn_partial_fused(ctypes.byref(p64), *([None] * 11), None) == dt.DT_ERR_UNSUPPORTED
+    p64.P = 64
+    assert lib.dt_attn_partial_fused(ctypes.byref(p64), *([None] * 11), None) == dt.DT_ERR_INVALID  # null buffers
+    # misaligned device pointers (the plan included) are refused on the host
     p = dt.params(1, 128, 64, 1, dt.DT_MODE_ALL_COMPUTE, 0, 0, 1)
+    plan_fake = [16 * 1024 + 4] + [16 * 1024] * 9
+    assert lib.dt_attn_partial_fused(ctypes.byref(p), *plan_fake, 16 * 1024, None) == dt.DT_ERR_UNSUPPORTED
     fake = [16 * 1024] * 10
     fake[1] = 16 * 1024 + 2
     assert lib.dt_attn_partial_fused(ctypes.byref(p), *fake, 16 * 1024, None) == dt.DT_ERR_UNSUPPORTED

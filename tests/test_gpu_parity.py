@@ -138,6 +138,8 @@ def test_video_workload_full_size_sampled_rows():
     (3, 2000, 64, 7, 3),
     (1, 128, 72, 1, 0),       # one tile, one partition
     (2, 4100, 128, 2, 1),     # 33 key tiles per head, ragged tail of 4 rows
+    (1, 2600, 64, 64, 40),    # the most partitions the fused kernel takes (64-bit plan mask)
+    (1, 1800, 72, 12, 5),     # P not a multiple of 4: byte-wise plan rows
 ])
 def test_ragged_geometry(H, S, D, P, r):
     run_partition_schedule(H, S, D, P, proximity_schedule(3, r), stream_of(H, S, D, 0.05, seed=S),
