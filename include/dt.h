@@ -140,6 +140,21 @@ DT_API int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan,
                           void* O, float* L,
                           int64_t* d_counters, int32_t* d_status, void* stream);
 
+/* The same step restricted to heads [head_begin, head_begin + head_count):
+ * the arguments are those of dt_attn_partial_fused, with the buffers of all
+ * p->H heads (same layouts, same pointers); only the rows of the selected
+ * heads are read or written, and each is computed exactly as the whole-step
+ * launch computes it (bit-identical), so launches over disjoint head ranges
+ * that cover all heads equal one whole-step launch.  Lets a caller overlap
+ * the host<->device copies of some heads with the computation of others.
+ * The counters accumulate the selected heads only.  Errors: those of
+ * dt_attn_partial_fused, and DT_ERR_INVALID for a range outside [0, H).
+ * head_count = 0 launches nothing and returns DT_OK. */
+DT_API int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head_begin, int32_t head_count,
+                          const uint8_t* d_plan, const void* Q, const void* K, const void* V,
+                          float* cache_O, float* cache_L, float* R, void* O, float* L,
+                          int64_t* d_counters, int32_t* d_status, void* stream);
+
 /* N-way composition of states ("DiTango", composition of attention states,
  * Eq. 4): for every row, L = M + ln sum_n e^(L_n - M), M = max_n L_n,
  * OUT = sum_n e^(L_n - L) OUT_n; rows whose N inputs are all empty get

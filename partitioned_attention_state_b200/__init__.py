@@ -19,7 +19,7 @@ import numpy as np
 
 __all__ = [
     "DtError", "PlanParams", "Plan", "lib_path", "load", "dt_status_string",
-    "dt_plan_geometry", "dt_plan_build", "dt_attn_partial_fused", "dt_state_merge",
+    "dt_plan_geometry", "dt_plan_build", "dt_attn_partial_fused", "dt_attn_partial_fused_heads", "dt_state_merge",
     "dt_state_cache_update", "dt_window_residual", "dt_set_wait_limit_ns",
     "DT_OK", "DT_ERR_INVALID", "DT_ERR_UNSUPPORTED", "DT_ERR_CACHE_EMPTY", "DT_ERR_CUDA",
     "DT_ERR_TIMEOUT", "DT_MODE_ALL_COMPUTE", "DT_MODE_PROXIMITY", "DT_MODE_ALL_REUSE",
@@ -75,6 +75,7 @@ def load() -> ctypes.CDLL:
             "dt_plan_geometry": ([pp, ctypes.POINTER(i32), ctypes.POINTER(i32)], ctypes.c_int),
             "dt_plan_build": ([pp, vp, ctypes.POINTER(Plan)], ctypes.c_int),
             "dt_attn_partial_fused": ([pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_attn_partial_fused_heads": ([pp, i32, i32] + [vp] * 12, ctypes.c_int),
             "dt_state_merge": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_state_cache_update": ([pp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_window_residual": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
@@ -145,6 +146,14 @@ def dt_attn_partial_fused(p: PlanParams, d_plan, Q, K, V, cache_O, cache_L, R, O
     _check(load().dt_attn_partial_fused(ctypes.byref(p), _ptr(d_plan), _ptr(Q), _ptr(K), _ptr(V), _ptr(cache_O),
                                         _ptr(cache_L), _ptr(R), _ptr(O), _ptr(L), _ptr(d_counters),
                                         _ptr(d_status), _stream(stream)), "dt_attn_partial_fused")
+
+
+def dt_attn_partial_fused_heads(p: PlanParams, head_begin: int, head_count: int, d_plan, Q, K, V, cache_O, cache_L,
+                                R, O, L, d_counters, d_status, stream=None) -> None:
+    _check(load().dt_attn_partial_fused_heads(ctypes.byref(p), head_begin, head_count, _ptr(d_plan), _ptr(Q), _ptr(K),
+                                              _ptr(V), _ptr(cache_O), _ptr(cache_L), _ptr(R), _ptr(O), _ptr(L),
+                                              _ptr(d_counters), _ptr(d_status), _stream(stream)),
+           "dt_attn_partial_fused_heads")
 
 
 def dt_state_merge(N, H, S, D, O_in, L_in, O_out, L_out, d_status=None, stream=None) -> None:

@@ -74,16 +74,18 @@ extern "C" int dt_set_wait_limit_ns(int64_t ns) {
   return DT_OK;
 }
 
-extern "C" int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan, const void* Q, const void* K,
-                                     const void* V, float* cache_O, float* cache_L, float* R, void* O, float* L,
-                                     int64_t* d_counters, int32_t* d_status, void* stream) {
+extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head_begin, int32_t head_count,
+                                           const uint8_t* d_plan, const void* Q, const void* K, const void* V,
+                                           float* cache_O, float* cache_L, float* R, void* O, float* L,
+                                           int64_t* d_counters, int32_t* d_status, void* stream) {
   if (!p || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW) return DT_ERR_INVALID;
   const bool win = p->mode == DT_MODE_WINDOW;
   if (!shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (win ? p->window < 1 : p->P < 1) return DT_ERR_INVALID;
+  if (head_begin < 0 || head_count < 0 || head_begin > p->H - head_count) return DT_ERR_INVALID;
   if (p->D != 64 && p->D != 72 && p->D != 128) return DT_ERR_UNSUPPORTED;
   if (!win && p->P > 64) return DT_ERR_UNSUPPORTED;      // the kernel keeps a plan row as a 64-bit mask
-  if (p->H == 0 || p->S == 0) return DT_OK;
+  if (head_count == 0 || p->S == 0) return DT_OK;
   if (!d_plan || !Q || !K || !V || !O || !L || !d_status) return DT_ERR_INVALID;
   if (win ? !R : (!cache_O || !cache_L)) return DT_ERR_INVALID;
   const void* ptrs[] = {d_plan, Q, K, V, O, L, d_status};
@@ -116,13 +118,26 @@ extern "C" int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_p
   kp.status = d_status;
   kp.H = p->H; kp.S = p->S; kp.D = p->D; kp.P = win ? 1 : p->P; kp.window = win ? p->window : 0;
   kp.geom = G;
-  kp.n_items = p->H * G.nqt;
+  // items are numbered over all heads, so a head range computes exactly what
+  // the whole launch computes for those heads
+  kp.item0 = head_begin * G.nqt;
+  kp.item_end = (head_begin + head_count) * G.nqt;
   kp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->D));
   kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
   int sms = 0;
   if (int e = sm_count(&sms)) return e;
-  int grid = kp.n_items < sms ? kp.n_items : sms;
+  const int n_items = kp.item_end - kp.item0;
+  if (n_items == 0) return DT_OK;
+  int grid = n_items < sms ? n_items : sms;
   return dt::launch_attn_fused(kp, dp, grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan, const void* Q, const void* K,
+                                     const void* V, float* cache_O, float* cache_L, float* R, void* O, float* L,
+                                     int64_t* d_counters, int32_t* d_status, void* stream) {
+  if (!p) return DT_ERR_INVALID;
+  return dt_attn_partial_fused_heads(p, 0, p->H, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,
+                                     stream);
 }
 
 extern "C" int dt_state_merge(int32_t N, int32_t H, int32_t S, int32_t D, const float* O_in, const float* L_in,

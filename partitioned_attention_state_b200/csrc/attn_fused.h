@@ -22,7 +22,7 @@ struct AttnParams {
   int32_t* status;
   int H, S, D, P, window;           // P: partitions (ignored in window mode)
   Geom geom;                        // make_geom(H, S, D, P, window), read from the parameter bank
-  int n_items;                      // H * nqt
+  int item0, item_end;              // items [item0, item_end) of the H * nqt (head-major) items
   float scale_log2;                 // log2(e) / sqrt(D)
   uint64_t wait_limit_ns;
 };

@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       // against the streaming state-cache traffic; a Q tile is read once.
       const uint64_t pol_keep = l2_policy_evict_last(), pol_once = l2_policy_evict_first();
       uint32_t g = 0, nq = 0;
-      for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+      for (int idx = p.item0 + blockIdx.x; idx < p.item_end; idx += gridDim.x) {
         const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       uint32_t g = 0, nq = 0;
       bool ok = true;
 
-      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+      for (int idx = p.item0 + blockIdx.x; idx < p.item_end && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const uint32_t aV = smem_u32(sV);
       uint32_t g = 0, cseg = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+      for (int idx = p.item0 + blockIdx.x; idx < p.item_end && ok; idx += gridDim.x) {
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
@@ -474,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     const uint32_t lane_base = static_cast<uint32_t>(rbase) << 16;
     const float sl2 = p.scale_log2;
     uint32_t g = 0, cseg = 0;
-    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+    for (int idx = p.item0 + blockIdx.x; idx < p.item_end; idx += gridDim.x) {
       const int qt = idx - (idx / G.nqt) * G.nqt;
       const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
       const int rot = seg_rotation<WIN>(G, idx);
@@ -661,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     float* orow = sO + r;
     uint32_t cseg = 0;
     uint32_t n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
-    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+    for (int idx = p.item0 + blockIdx.x; idx < p.item_end; idx += gridDim.x) {
       const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
       const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
       const int rot = seg_rotation<WIN>(G, idx);

@@ -3,8 +3,10 @@
 A ``Session`` owns the device tensors of one workload (inputs, state cache,
 residual, outputs, counters, status word) and the host stamps, and runs one
 denoising step as: host plan build (``dt_plan_build``) -> plan upload ->
-one fused launch (``dt_attn_partial_fused``).  torch provides the memory and
-the stream; every computation happens in libdt.
+one fused launch (``dt_attn_partial_fused``), or, from host buffers, as
+head-group launches (``dt_attn_partial_fused_heads``) pipelined with their
+copies.  torch provides the memory and the streams; every computation
+happens in libdt.
 """
 
 from __future__ import annotations
@@ -14,8 +16,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused, dt_plan_build, dt_plan_geometry, DtError,
-               params)
+from . import (DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused, dt_attn_partial_fused_heads, dt_plan_build,
+               dt_plan_geometry, DtError, params)
 
 
 def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
@@ -81,20 +83,81 @@ class Session:
              stream=None) -> dict:
         """Host plan build, asynchronous plan upload, one fused launch."""
         p, plan, counts = self.plan(step, mode, explicit)
-        if self.nqt > 0:
-            i = self._turn
-            self._turn ^= 1
-            if self._uploaded[i] is not None:
-                self._uploaded[i].synchronize()      # that buffer's previous upload is done
-            buf = self._pinned[i]
-            buf[: self.nqt].numpy()[...] = plan
-            st = torch.cuda.current_stream(self.device) if stream is None else stream
-            with torch.cuda.stream(st):
-                self.d_plan[: self.nqt].copy_(buf[: self.nqt], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(st)
-            self._uploaded[i] = ev
+        self._upload_plan(plan, torch.cuda.current_stream(self.device) if stream is None else stream)
         self.launch(p, stream)
+        self.last_counts, self.last_plan = counts, plan
+        return counts
+
+    def _upload_plan(self, plan: np.ndarray, st) -> None:
+        """Asynchronous copy of a host plan into d_plan, ordered on stream `st`."""
+        if self.nqt == 0:
+            return
+        i = self._turn
+        self._turn ^= 1
+        if self._uploaded[i] is not None:
+            self._uploaded[i].synchronize()      # that buffer's previous upload is done
+        buf = self._pinned[i]
+        buf[: self.nqt].numpy()[...] = plan
+        with torch.cuda.stream(st):
+            self.d_plan[: self.nqt].copy_(buf[: self.nqt], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(st)
+        self._uploaded[i] = ev
+
+    def step_host(self, step: int, q, k, v, o, lse, groups: Optional[int] = None, mode: Optional[int] = None,
+                  explicit: Optional[np.ndarray] = None) -> dict:
+        """One step from host inputs to host outputs.
+
+        q, k, v: pinned host tensors [H][S][D] of bf16 (or of 16-bit integers
+        holding bf16 bit patterns); o: pinned host [H][S][D] of the same kind,
+        lse: pinned host float32 [H][S].  The heads are split into `groups`
+        contiguous groups (default: one group per ~16 MB of inputs, at most
+        16 and at most H, since each group adds a launch and five copy
+        calls of fixed cost); group g is uploaded on one
+        stream, computed by a head-range fused launch on a second and
+        downloaded on a third, so the copies of one group overlap the
+        computation of the others.  Each head is computed exactly as a whole
+        step computes it.  The work is ordered after, and the current stream
+        made to wait for, everything issued here: synchronise the current
+        stream before reading o and lse.  Returns the plan counts."""
+        dev = self.device
+        cur = torch.cuda.current_stream(dev)
+        if getattr(self, "_host_streams", None) is None:
+            self._host_streams = tuple(torch.cuda.Stream(dev) for _ in range(3))
+        up, comp, down = self._host_streams
+        for st in self._host_streams:
+            st.wait_stream(cur)
+        p, plan, counts = self.plan(step, mode, explicit)
+        self._upload_plan(plan, comp)
+        H = self.H
+        if groups is None:
+            groups = min(16, (3 * q.numel() * q.element_size()) // (16 << 20))
+        n = max(1, min(H, int(groups)))
+        bounds = [H * g // n for g in range(n + 1)]
+
+        def dev_view(d, h):
+            return d if h.dtype == d.dtype else d.view(h.dtype)
+
+        for g in range(n):
+            h0, h1 = bounds[g], bounds[g + 1]
+            if h1 == h0:
+                continue
+            with torch.cuda.stream(up):
+                for d, h in ((self.Q, q), (self.K, k), (self.V, v)):
+                    dev_view(d, h)[h0:h1].copy_(h[h0:h1], non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(up)
+            comp.wait_event(arrived)
+            dt_attn_partial_fused_heads(p, h0, h1 - h0, self.d_plan, self.Q, self.K, self.V, self.cache_O,
+                                        self.cache_L, self.R, self.O, self.L, self.counters, self.status, comp)
+            done = torch.cuda.Event()
+            done.record(comp)
+            down.wait_event(done)
+            with torch.cuda.stream(down):
+                o[h0:h1].copy_(dev_view(self.O, o)[h0:h1], non_blocking=True)
+                lse[h0:h1].copy_(self.L[h0:h1], non_blocking=True)
+        for st in self._host_streams:
+            cur.wait_stream(st)
         self.last_counts, self.last_plan = counts, plan
         return counts
 

@@ -160,3 +160,18 @@ def test_device_entry_points_validate_before_any_cuda_call():
     fake = [16 * 1024] * 10
     fake[1] = 16 * 1024 + 2
     assert lib.dt_attn_partial_fused(ctypes.byref(p), *fake, 16 * 1024, None) == dt.DT_ERR_UNSUPPORTED
+
+
+def test_head_range_validated_on_the_host():
+    """dt_attn_partial_fused_heads refuses ranges outside [0, H) before any
+    CUDA call; an empty range launches nothing."""
+    import ctypes
+    lib = dt.load()
+    p = dt.params(3, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1)
+    for h0, n in ((-1, 1), (0, -1), (1, 3), (3, 1), (0, 4)):
+        assert lib.dt_attn_partial_fused_heads(ctypes.byref(p), h0, n, *([None] * 11), None) == dt.DT_ERR_INVALID
+    for h0 in (0, 2, 3):
+        assert lib.dt_attn_partial_fused_heads(ctypes.byref(p), h0, 0, *([None] * 11), None) == dt.DT_OK
+    # a valid range still needs its buffers
+    assert lib.dt_attn_partial_fused_heads(ctypes.byref(p), 1, 2, *([None] * 11), None) == dt.DT_ERR_INVALID
+    assert lib.dt_attn_partial_fused_heads(None, 0, 1, *([None] * 11), None) == dt.DT_ERR_INVALID

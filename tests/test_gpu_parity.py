@@ -248,3 +248,63 @@ def test_graph_replay_matches_eager_step():
     sess.check()
     assert torch.equal(sess.O.view(torch.int16), o_eager.view(torch.int16))
     assert torch.equal(sess.L, l_eager)
+
+
+def _pinned_like(t, dtype=None):
+    return torch.empty(t.shape, dtype=t.dtype if dtype is None else dtype).pin_memory()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,groups", [("dit_xl2_512_32x32_h16_d72_p8", 3), ("tiny_4x16x16_h2_d64_p4", 8),
+                                         ("dit_xl2_512_32x32_h16_d72_p8", 1)])
+def test_host_step_head_groups_match_whole_step(name, groups):
+    """Session.step_host (head-range launches pipelined with their copies)
+    writes the same bytes as the whole-step launch: same outputs, same cache
+    slots, same counters."""
+    w = wl.BY_NAME[name]
+    s = wl.stream_for(w)
+    steps = [s.next_step() for _ in range(3)]
+    a = Session(w.H, w.S, w.D, w.P, reuse_per_row=w.P // 2)
+    b = Session(w.H, w.S, w.D, w.P, reuse_per_row=w.P // 2)
+    ho = _pinned_like(b.O, torch.int16)
+    hl = _pinned_like(b.L)
+    for t, (q, k, v) in enumerate(steps, start=1):
+        a.set_inputs(q, k, v)
+        a.counters.zero_()
+        ca = a.step(t)
+        a.check()
+        hq = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in (q, k, v)]
+        b.counters.zero_()
+        cb = b.step_host(t, *hq, ho, hl, groups=groups)
+        torch.cuda.current_stream().synchronize()
+        b.check()
+        assert ca == cb
+        assert torch.equal(a.counters, b.counters)
+        assert torch.equal(a.O.view(torch.int16).cpu(), ho)
+        assert torch.equal(a.L.cpu(), hl)
+        assert torch.equal(a.cache_O, b.cache_O) and torch.equal(a.cache_L, b.cache_L)
+
+
+@pytest.mark.gpu
+def test_host_step_window_mode_matches_whole_step():
+    """Window mode through step_host: anchor step (writes R) and two residual
+    steps, byte-identical to whole-step launches."""
+    w = wl.BY_NAME["window_128x128_h16_d72_w1024"]
+    H, S = 4, 4096
+    s = wl.InputStream(H, S, w.D, w.sigma, seed=3)
+    a = Session(H, S, w.D, mode=dt.DT_MODE_WINDOW, window=w.window)
+    b = Session(H, S, w.D, mode=dt.DT_MODE_WINDOW, window=w.window)
+    ho = _pinned_like(b.O, torch.int16)
+    hl = _pinned_like(b.L)
+    for t in (1, 2, 3):
+        q, k, v = s.next_step()
+        a.set_inputs(q, k, v)
+        a.step(t)
+        a.check()
+        hq = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in (q, k, v)]
+        b.step_host(t, *hq, ho, hl, groups=3)
+        torch.cuda.current_stream().synchronize()
+        b.check()
+        assert torch.equal(a.O.view(torch.int16).cpu(), ho)
+        assert torch.equal(a.L.cpu(), hl)
+        assert torch.equal(a.R, b.R)
