@@ -27,7 +27,17 @@ notes of the repository):
     are reused, ties broken towards the lower index; q itself is always
     computed; step 1 is an anchor (everything computed);
   * window: key j is in the window of query i iff |i - j| <= W // 2 on the
-    flattened token order, no wrap-around.
+    flattened token order, no wrap-around;
+  * state grouping with group size g: groups of g adjacent partitions,
+    G_i = [i g, min((i+1) g, P)); a query in partition q has the key sets
+    {q} (its local state, handled separately) and G_i without q for every i
+    (the group holding q keeps g - 1 partitions); one composed state is
+    cached per (query tile, key set) and the plan decides per key set; the
+    proximity plan reuses the r groups farthest from q's group (lower index
+    first among equal distances) and always computes {q};
+  * Dynamic Group State Compose by a factor k: the new group i is old groups
+    k i .. k i + k - 1, its cached state their composition, its stamp the
+    oldest of theirs (never written if any was never written).
 """
 
 from __future__ import annotations
@@ -54,6 +64,8 @@ __all__ = [
     "attention_state", "identity_state", "compose", "compose_n",
     "proximity_row", "build_plan", "window_in", "StateCache",
     "partition_step", "window_step", "softmax_scale",
+    "n_groups", "group_key_sets", "group_proximity_row", "key_sets_of_tile",
+    "compose_groups",
 ]
 
 
@@ -231,14 +243,49 @@ def _window_pairs(q0: int, q1: int, S: int, W: int) -> int:
     return tot
 
 
+def n_groups(P: int, g: int) -> int:
+    """[DT] grouping: m = ceil(P / g) groups of g adjacent partitions."""
+    return -(-P // g)
+
+
+def group_key_sets(q: int, P: int, g: int) -> List[List[int]]:
+    """[DT] grouping: key sets of a query in partition q, as lists of
+    partitions.  Set 0 is the local partition {q}; set 1 + i is group
+    G_i = partitions [i g, min((i+1) g, P)) without q, so the group that
+    holds q has g - 1 partitions (none when g = 1)."""
+    sets = [[q]]
+    for i in range(n_groups(P, g)):
+        sets.append([k for k in range(i * g, min((i + 1) * g, P)) if k != q])
+    return sets
+
+
+def group_proximity_row(q: int, P: int, g: int, r: int) -> np.ndarray:
+    """Plan row over the 1 + m key sets of a query in partition q: the local
+    set is always computed; the r groups farthest from q's group q // g are
+    reused, lower index first among equal distances."""
+    m = n_groups(P, g)
+    row = np.full(1 + m, COMPUTE, dtype=np.uint8)
+    lg = q // g
+    for i in sorted(range(m), key=lambda i: (-abs(i - lg), i))[:r]:
+        row[1 + i] = REUSE
+    return row
+
+
+def key_sets_of_tile(q: int, P: int, group: int) -> List[List[int]]:
+    """Key sets (lists of partitions) of a query tile in partition q: one per
+    partition without grouping (group = 0), else the grouped sets."""
+    return [[k] for k in range(P)] if group == 0 else group_key_sets(q, P, group)
+
+
 def build_plan(mode: int, H: int, S: int, D: int, P: int, step: int,
                r: int = 0, window: int = 0,
                stamps: Optional[np.ndarray] = None,
-               explicit: Optional[np.ndarray] = None):
+               explicit: Optional[np.ndarray] = None, group: int = 0):
     """Plan, block counts, algorithmic FLOPs and updated stamps of one step.
 
     Returns ``(plan uint8 [nqt][nseg], counts, stamps')`` where nseg = P (2 in
-    window mode: key sets "window" and "complement"), counts =
+    window mode: key sets "window" and "complement"; 1 + ceil(P / group) with
+    grouping, where r counts groups), counts =
     {computed_blocks, skipped_blocks, computed_flops}.  Step 1 of the proximity
     and window modes is an anchor: everything is computed.  A REUSE entry whose
     stamp is -1 raises ``CacheEmpty``; COMPUTE entries get stamp = step.
@@ -251,17 +298,17 @@ def build_plan(mode: int, H: int, S: int, D: int, P: int, step: int,
         if step > 1:
             plan[:, 1] = REUSE
     else:
-        nseg = P
-        plan = np.empty((nqt, P), dtype=np.uint8)
+        nseg = P if group == 0 else 1 + n_groups(P, group)
+        plan = np.empty((nqt, nseg), dtype=np.uint8)
         for t, (kq, _, _) in enumerate(tiles):
             if mode == MODE_ALL_COMPUTE or (mode == MODE_PROXIMITY and step <= 1):
                 plan[t] = COMPUTE
             elif mode == MODE_PROXIMITY:
-                plan[t] = proximity_row(kq, P, r)
+                plan[t] = proximity_row(kq, P, r) if group == 0 else group_proximity_row(kq, P, group, r)
             elif mode == MODE_ALL_REUSE:
                 plan[t] = REUSE
             elif mode == MODE_EXPLICIT:
-                plan[t] = np.asarray(explicit, dtype=np.uint8).reshape(nqt, P)[t]
+                plan[t] = np.asarray(explicit, dtype=np.uint8).reshape(nqt, nseg)[t]
             else:
                 raise ValueError(mode)
     st = (np.full((nqt, nseg), -1, dtype=np.int32) if stamps is None
@@ -283,11 +330,12 @@ def build_plan(mode: int, H: int, S: int, D: int, P: int, step: int,
                 sb += H * (nkt - band)
                 fl += 4 * H * D * _window_pairs(q0, q1, S, window)
         else:
-            for k, (a, b) in enumerate(parts):
-                nb = H * n_kv_tiles(a, b)
+            kq = tiles[t][0]
+            for k, ks in enumerate(key_sets_of_tile(kq, P, group)):
+                nb = H * sum(n_kv_tiles(*parts[j]) for j in ks)
                 if plan[t, k] == COMPUTE:
                     cb += nb
-                    fl += 4 * H * D * (q1 - q0) * (b - a)
+                    fl += 4 * H * D * (q1 - q0) * sum(parts[j][1] - parts[j][0] for j in ks)
                 else:
                     sb += nb
     counts = {"computed_blocks": cb, "skipped_blocks": sb, "computed_flops": fl}
@@ -330,9 +378,12 @@ def _tile_of_rows(tiles, rows):
 def partition_step(Q: np.ndarray, K: np.ndarray, V: np.ndarray, plan: np.ndarray,
                    S: int, P: int, cache: StateCache,
                    heads: Optional[Sequence[int]] = None,
-                   rows: Optional[np.ndarray] = None):
+                   rows: Optional[np.ndarray] = None, group: int = 0):
     """[DT] One step: (O, LSE)_q = compose over k of (fresh if COMPUTE else
-    cached); fresh states overwrite their slots afterwards.
+    cached); fresh states overwrite their slots afterwards.  Key set k is
+    partition k, or with grouping (group > 0) the k-th grouped key set of the
+    query's partition; the state of a set is the attention state over the
+    union of its partitions' keys.
 
     Q, K, V: float64 [H][S][D] (or bf16 bits, widened here).  Returns
     ``(O, LSE, fresh)`` for the selected heads x rows, O in float64 (the
@@ -357,9 +408,11 @@ def partition_step(Q: np.ndarray, K: np.ndarray, V: np.ndarray, plan: np.ndarray
             sel = np.nonzero(tix == t)[0]
             rs = rows[sel]
             states = []
-            for k, (a, b) in enumerate(parts):
+            for k, ks in enumerate(key_sets_of_tile(tiles[t][0], P, group)):
                 if plan[t, k] == COMPUTE:
-                    st = attention_state(Q[h, rs], K[h, a:b], V[h, a:b], scale)
+                    keys = np.concatenate([np.arange(*parts[j]) for j in ks]).astype(np.int64) if ks else \
+                        np.zeros(0, dtype=np.int64)
+                    st = attention_state(Q[h, rs], K[h, keys], V[h, keys], scale)
                     pending.append((k, h, rs, st))
                     fresh.setdefault((k, h), []).append((rs, st))
                 else:
@@ -372,6 +425,43 @@ def partition_step(Q: np.ndarray, K: np.ndarray, V: np.ndarray, plan: np.ndarray
         for k, h_, rs, st in pending:
             cache.put(k, h_, rs, st[0], st[1])
     return O, L, fresh
+
+
+def _get_or_identity(cache: StateCache, k, h, rs, D):
+    """A slot never written holds nothing; its stamp (-1) already marks the
+    composed slot unusable, so the identity stands in for its content."""
+    try:
+        return cache.get(k, h, rs, D)
+    except KeyError:
+        return identity_state(len(rs), D)
+
+
+def compose_groups(cache: StateCache, stamps: np.ndarray, P: int, g: int, kf: int,
+                   heads: Sequence[int], rows: np.ndarray, S: int, D: int):
+    """[DT] Dynamic Group State Compose: regroup the cached states of group
+    size g into group size kf * g.  New set 0 is old set 0; new set 1 + i is
+    the composition of old sets 1 + j, j = kf i .. min(kf i + kf, m) - 1.  The
+    new stamp is the oldest of the merged stamps (-1 if any is -1).  Returns
+    ``(new cache, new stamps)`` for the tracked heads x rows."""
+    m, m2 = n_groups(P, g), n_groups(P, kf * g)
+    new = StateCache()
+    tiles = query_tiles(S, P)
+    tix = _tile_of_rows(tiles, np.asarray(rows))
+    for h in heads:
+        for t in np.unique(tix):
+            rs = np.asarray(rows)[tix == t]
+            o, l = cache.get(0, h, rs, D)
+            new.put(0, h, rs, o, l)
+            for i in range(m2):
+                merged = [_get_or_identity(cache, 1 + j, h, rs, D) for j in range(kf * i, min(kf * i + kf, m))]
+                o, l = compose_n(merged)
+                new.put(1 + i, h, rs, o, l)
+    st = np.asarray(stamps).reshape(-1, 1 + m)
+    st2 = np.empty((st.shape[0], 1 + m2), dtype=np.int32)
+    st2[:, 0] = st[:, 0]
+    for i in range(m2):
+        st2[:, 1 + i] = st[:, 1 + kf * i: 1 + min(kf * i + kf, m)].min(axis=1)
+    return new, st2
 
 
 def window_step(Q: np.ndarray, K: np.ndarray, V: np.ndarray, W: int,
