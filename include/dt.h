@@ -28,11 +28,12 @@
  *   - tensors are dense, row-major, batch 1:
  *       Q, K, V, O           bf16  [H][S][D]
  *       L (final LSE)        fp32  [H][S]
- *       cache_O              fp32  [P][H][S][D]   (state OUT of partition k)
- *       cache_L              fp32  [P][H][S]      (state LSE of partition k)
+ *       cache_O              fp32  [nseg][H][S][D] (state OUT of key set k)
+ *       cache_L              fp32  [nseg][H][S]    (state LSE of key set k)
  *       R (window residual)  fp32  [H][S][D]
- *     The state of query row s, head h, KV partition k lives at
- *     cache_O[((k*H + h)*S + s)*D + d] and cache_L[(k*H + h)*S + s].
+ *     The state of query row s, head h, key set k (KV partition k, or the
+ *     k-th grouped key set) lives at cache_O[((k*H + h)*S + s)*D + d] and
+ *     cache_L[(k*H + h)*S + s]; nseg = P without grouping.
  *   - softmax scale is 1/sqrt(D); LSE is a natural logarithm; OUT is
  *     normalised by the partition's own softmax denominator.
  */
@@ -76,10 +77,23 @@ extern "C" {
 typedef struct {
   int32_t H, S, D, P;           /* heads, tokens, head dim, partitions (P ignored in window mode) */
   int32_t mode;                 /* DT_MODE_* */
-  int32_t reuse_per_row;        /* r: partitions reused per query partition (proximity) */
+  int32_t reuse_per_row;        /* r: partitions (with grouping: groups) reused per query partition (proximity) */
   int32_t window;               /* W: key j is in query i's window iff |i-j| <= W/2 (window mode) */
   int32_t step;                 /* denoising step t, 1-based; step 1 is an anchor */
+  int32_t group;                /* g: 0 = one key set per partition; g >= 1 = state grouping (below).
+                                   Partition modes only (0 in window mode) */
 } dt_plan_params;
+
+/* State grouping ("DiTango", grouping of spatially adjacent attention states;
+ * the local state is handled separately): with group size g the P partitions
+ * form m = ceil(P/g) groups G_i = partitions [i*g, min((i+1)*g, P)).  A query
+ * tile of partition q then has nseg = 1 + m key sets: set 0 = {q}, set 1+i =
+ * G_i without q (the group holding q keeps g-1 partitions, none if g = 1).
+ * One state per (query tile, key set) is computed or reused and cached: a
+ * group's slot holds the composition of its partitions' states.  The
+ * proximity plan always computes set 0 and reuses the r groups farthest from
+ * q's group q/g (|i - q/g|, equal distances lower index first; r <= m).
+ * nseg must not exceed 64 for the fused kernel. */
 
 typedef struct {
   uint8_t* plan;                /* caller-allocated host [nqt][nseg] (out) */
@@ -89,7 +103,8 @@ typedef struct {
   int64_t skipped_blocks;       /* (out) blocks covered by reused states, x H */
   int64_t computed_flops;       /* (out) 4*D*(query,key) pairs computed, x H */
   int32_t nqt;                  /* (out) query tiles per head */
-  int32_t nseg;                 /* (out) key sets per query tile: P, or 2 in window mode */
+  int32_t nseg;                 /* (out) key sets per query tile: P, 1 + ceil(P/g) with
+                                   grouping, or 2 in window mode */
 } dt_plan;
 
 /* Human-readable name of a status code (static storage, never NULL). */
@@ -115,13 +130,15 @@ DT_API int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, 
 
 /* Fused step on the GPU ("DiTango", attention state Eq. 1-3, composition Eq. 4,
  * selective reuse Fig. 6).  For each head and query tile and each key set of
- * the tile's plan row: COMPUTE runs the partial attention (tensor cores) and
+ * the tile's plan row (a partition, a group of partitions with p->group >= 1,
+ * or a window-mode set): COMPUTE runs the partial attention (tensor cores) and
  * writes the fresh state (OUT, LSE) to its cache slot; REUSE reads the cached
  * state.  All states of the row are composed into O (bf16) and L.
  *   d_plan      device copy of dt_plan.plan, [nqt][nseg] uint8
  *   Q, K, V     bf16 [H][S][D] (read)
- *   cache_O/L   state slots (REUSE slots read, COMPUTE slots written; slots of
- *               other pairs untouched).  May be NULL in window mode.
+ *   cache_O/L   fp32 [nseg][H][S][D] / [nseg][H][S] state slots, slot (k, h,
+ *               row) for key set k (REUSE slots read, COMPUTE slots written;
+ *               slots of other pairs untouched).  May be NULL in window mode.
  *   R           window mode only: fp32 [H][S][D]; written at the anchor step
  *               (R = OUT_full - OUT_window), read afterwards (O = OUT_window + R,
  *               L = LSE_window).  NULL otherwise.
@@ -132,7 +149,7 @@ DT_API int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, 
  *               counted per (query tile, key set, head)
  *   d_status    int32 device status word (see conventions)
  * The host validates shapes and alignment before any launch.  One launch.
- * Partition mode supports at most 64 partitions (DT_ERR_UNSUPPORTED above);
+ * Partition mode supports at most 64 key sets (DT_ERR_UNSUPPORTED above);
  * d_plan must be 16-byte aligned like every other pointer. */
 DT_API int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan,
                           const void* Q, const void* K, const void* V,
@@ -173,6 +190,21 @@ DT_API int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_plan,
                           const float* fresh_O, const float* fresh_L,
                           float* cache_O, float* cache_L,
                           int32_t* d_status, void* stream);
+
+/* Dynamic Group State Compose ("DiTango", merging cached states into
+ * k-times coarser groups, composability Eq. 4): regroups the cache of the
+ * grouped layout p (p->group = g >= 1, partition modes) into group size
+ * g*factor, in place.  New set 0 = old set 0; new set 1+i = composition of old
+ * sets 1+j, j = factor*i .. min(factor*i + factor, m) - 1.  Afterwards slots
+ * [0, 1 + ceil(m/factor)) of cache_O [nseg][H][S][D] / cache_L [nseg][H][S]
+ * hold the coarse layout (later slots are stale), and the caller continues
+ * with p->group = g*factor.  stamps (host, optional) is [nqt][1+m] on entry
+ * and is rewritten as [nqt][1+m'] in its first entries: a composed slot gets
+ * the oldest stamp of the slots it merges (-1 if any is -1).  One launch of an
+ * HBM-bound kernel.  Errors: DT_ERR_INVALID (bad params, factor < 2, null
+ * cache), DT_ERR_UNSUPPORTED (misaligned cache pointers). */
+DT_API int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t* stamps,
+                     float* cache_O, float* cache_L, int32_t* d_status, void* stream);
 
 #define DT_WR_MAKE  0   /* R = O_full - O_win                 */
 #define DT_WR_APPLY 1   /* O = bf16(O_win + R)  (O_full unused) */

@@ -20,7 +20,7 @@ import numpy as np
 __all__ = [
     "DtError", "PlanParams", "Plan", "lib_path", "load", "dt_status_string",
     "dt_plan_geometry", "dt_plan_build", "dt_attn_partial_fused", "dt_attn_partial_fused_heads", "dt_state_merge",
-    "dt_state_cache_update", "dt_window_residual", "dt_set_wait_limit_ns",
+    "dt_state_cache_update", "dt_group_compose", "dt_window_residual", "dt_set_wait_limit_ns",
     "DT_OK", "DT_ERR_INVALID", "DT_ERR_UNSUPPORTED", "DT_ERR_CACHE_EMPTY", "DT_ERR_CUDA",
     "DT_ERR_TIMEOUT", "DT_MODE_ALL_COMPUTE", "DT_MODE_PROXIMITY", "DT_MODE_ALL_REUSE",
     "DT_MODE_EXPLICIT", "DT_MODE_WINDOW", "DT_PLAN_REUSE", "DT_PLAN_COMPUTE", "DT_WR_MAKE",
@@ -43,7 +43,7 @@ class DtError(RuntimeError):
 class PlanParams(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int32), ("S", ctypes.c_int32), ("D", ctypes.c_int32), ("P", ctypes.c_int32),
                 ("mode", ctypes.c_int32), ("reuse_per_row", ctypes.c_int32), ("window", ctypes.c_int32),
-                ("step", ctypes.c_int32)]
+                ("step", ctypes.c_int32), ("group", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):
@@ -79,6 +79,7 @@ def load() -> ctypes.CDLL:
             "dt_state_merge": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_state_cache_update": ([pp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_window_residual": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_group_compose": ([pp, i32, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_set_wait_limit_ns": ([i64], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -113,8 +114,8 @@ def dt_status_string(status: int) -> str:
     return load().dt_status_string(status).decode()
 
 
-def params(H, S, D, P=1, mode=DT_MODE_ALL_COMPUTE, reuse_per_row=0, window=0, step=1) -> PlanParams:
-    return PlanParams(H, S, D, P, mode, reuse_per_row, window, step)
+def params(H, S, D, P=1, mode=DT_MODE_ALL_COMPUTE, reuse_per_row=0, window=0, step=1, group=0) -> PlanParams:
+    return PlanParams(H, S, D, P, mode, reuse_per_row, window, step, group)
 
 
 def dt_plan_geometry(p: PlanParams):
@@ -154,6 +155,23 @@ def dt_attn_partial_fused_heads(p: PlanParams, head_begin: int, head_count: int,
                                               _ptr(V), _ptr(cache_O), _ptr(cache_L), _ptr(R), _ptr(O), _ptr(L),
                                               _ptr(d_counters), _ptr(d_status), _stream(stream)),
            "dt_attn_partial_fused_heads")
+
+
+def dt_group_compose(p: PlanParams, factor: int, stamps: Optional[np.ndarray], cache_O, cache_L, d_status=None,
+                     stream=None) -> Optional[np.ndarray]:
+    """Regroup the cached states of layout p (p.group = g) into group size
+    g * factor in place.  ``stamps`` (int32 [nqt][1+m], host) is rewritten in
+    place; the returned view is its new [nqt][1+m'] shape (None if None)."""
+    if stamps is not None:
+        assert stamps.dtype == np.int32 and stamps.flags.c_contiguous
+    _check(load().dt_group_compose(ctypes.byref(p), factor, _ptr(stamps), _ptr(cache_O), _ptr(cache_L),
+                                   _ptr(d_status), _stream(stream)), "dt_group_compose")
+    if stamps is None:
+        return None
+    nqt = stamps.shape[0]
+    m = -(-p.P // p.group)
+    m2 = -(-m // factor)
+    return stamps.reshape(-1)[: nqt * (1 + m2)].reshape(nqt, 1 + m2)
 
 
 def dt_state_merge(N, H, S, D, O_in, L_in, O_out, L_out, d_status=None, stream=None) -> None:

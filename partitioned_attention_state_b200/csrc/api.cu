@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <cstring>
+#include <vector>
 
 #include "../../include/dt.h"
 #include "attn_fused.h"
@@ -82,9 +83,11 @@ extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head
   const bool win = p->mode == DT_MODE_WINDOW;
   if (!shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (win ? p->window < 1 : p->P < 1) return DT_ERR_INVALID;
+  if (p->group < 0 || (win && p->group != 0)) return DT_ERR_INVALID;
   if (head_begin < 0 || head_count < 0 || head_begin > p->H - head_count) return DT_ERR_INVALID;
   if (p->D != 64 && p->D != 72 && p->D != 128) return DT_ERR_UNSUPPORTED;
-  if (!win && p->P > 64) return DT_ERR_UNSUPPORTED;      // the kernel keeps a plan row as a 64-bit mask
+  const int nseg = win ? 2 : (p->group > 0 ? 1 + dt::ceil_div(p->P, p->group) : p->P);
+  if (nseg > 64) return DT_ERR_UNSUPPORTED;              // the kernel keeps a plan row as a 64-bit mask
   if (head_count == 0 || p->S == 0) return DT_OK;
   if (!d_plan || !Q || !K || !V || !O || !L || !d_status) return DT_ERR_INVALID;
   if (win ? !R : (!cache_O || !cache_L)) return DT_ERR_INVALID;
@@ -95,7 +98,7 @@ extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head
       (d_counters && !aligned16(d_counters)))
     return DT_ERR_UNSUPPORTED;
 
-  dt::Geom G = dt::make_geom(p->H, p->S, p->D, win ? 1 : p->P, win ? p->window : 0);
+  dt::Geom G = dt::make_geom(p->H, p->S, p->D, win ? 1 : p->P, win ? p->window : 0, win ? 0 : p->group);
   const int dp = p->D == 72 ? 80 : p->D;
   dt::AttnParams kp;
   memset(&kp, 0, sizeof(kp));
@@ -158,17 +161,53 @@ extern "C" int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_p
                                      void* stream) {
   if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW)
     return DT_ERR_INVALID;
-  if (p->P < 1 || p->D < 4 || p->D % 4 != 0 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
+  if (p->P < 1 || p->group < 0 || p->D < 4 || p->D % 4 != 0 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (p->H == 0 || p->S == 0) return DT_OK;
   if (!d_plan || !fresh_O || !fresh_L || !cache_O || !cache_L) return DT_ERR_INVALID;
   if (!aligned16(fresh_O) || !aligned16(cache_O) || !aligned16(fresh_L) || !aligned16(cache_L))
     return DT_ERR_UNSUPPORTED;
   (void)d_status;
-  dt::Geom G = dt::make_geom(p->H, p->S, p->D, p->P, 0);
+  dt::Geom G = dt::make_geom(p->H, p->S, p->D, p->P, 0, p->group);
   int sms = 0;
   if (int e = sm_count(&sms)) return e;
   return dt::launch_cache_update(G, d_plan, fresh_O, fresh_L, cache_O, cache_L, sms,
                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t* stamps, float* cache_O,
+                                float* cache_L, int32_t* d_status, void* stream) {
+  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW)
+    return DT_ERR_INVALID;
+  if (p->P < 1 || p->group < 1 || factor < 2 || factor > 8) return DT_ERR_INVALID;
+  if (p->D < 4 || p->D % 4 != 0 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
+  if ((int64_t)p->group * factor > (int64_t)1 << 30) return DT_ERR_INVALID;
+  const dt::Geom G = dt::make_geom(p->H, p->S, p->D, p->P, 0, p->group);
+  const int m = G.P - 1, m2 = dt::ceil_div(m, factor);
+  if ((int64_t)p->H * p->S > 0) {
+    if (!cache_O || !cache_L) return DT_ERR_INVALID;
+    if (!aligned16(cache_O) || !aligned16(cache_L)) return DT_ERR_UNSUPPORTED;
+  }
+  (void)d_status;
+  if (stamps) {
+    // [nqt][1+m] -> [nqt][1+m2] in place, row by row (a new row never starts
+    // after its old row, and each new row is built before it is written)
+    std::vector<int32_t> tmp(1 + m2);
+    for (int qt = 0; qt < G.nqt; ++qt) {
+      const int32_t* old_row = stamps + (size_t)qt * (1 + m);
+      tmp[0] = old_row[0];
+      for (int i = 0; i < m2; ++i) {
+        int32_t s = old_row[1 + factor * i];
+        for (int j = factor * i + 1; j < factor * i + factor && j < m; ++j) s = old_row[1 + j] < s ? old_row[1 + j] : s;
+        tmp[1 + i] = s;
+      }
+      memcpy(stamps + (size_t)qt * (1 + m2), tmp.data(), sizeof(int32_t) * (1 + m2));
+    }
+  }
+  if ((int64_t)p->H * p->S == 0) return DT_OK;
+  int sms = 0;
+  if (int e = sm_count(&sms)) return e;
+  return dt::launch_group_compose(m, factor, p->H, p->S, p->D, cache_O, cache_L, sms,
+                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int dt_window_residual(int32_t op, int32_t H, int32_t S, int32_t D, const float* O_full,

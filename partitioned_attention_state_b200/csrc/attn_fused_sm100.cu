@@ -8,6 +8,8 @@
 //   composition of states (Eq. 4), applied over all P partitions of a row;
 //   selective compute/reuse (Fig. 6): per (query tile, partition) the plan says
 //   COMPUTE (fresh state, written to its cache slot) or REUSE (cached state).
+//   With state grouping (grouping of adjacent states) a key set is a group of
+//   partitions instead of one, and its slot holds the group's composed state.
 // Window mode ("DiTFastAttn: Attention Compression for Diffusion Transformer
 // Models", window attention with residual sharing): key sets "window" and
 // "complement"; at the anchor step both are computed and R = OUT_full -
@@ -177,10 +179,10 @@ __device__ __forceinline__ uint64_t plan_mask(const uint8_t* prow, int P) {
 }
 __device__ __forceinline__ bool is_compute(uint64_t cm, int seg) { return (cm >> seg) & 1u; }
 
-template <bool WIN>
+template <int MODE>
 __device__ __forceinline__ bool item_has_compute(const Geom& G, int qt, uint64_t cm) {
   for (int s = 0; s < G.P; ++s)
-    if (is_compute(cm, s) && key_set<WIN>(G, qt, s).ntiles() > 0) return true;
+    if (is_compute(cm, s) && key_set<MODE>(G, qt, s).ntiles() > 0) return true;
   return false;
 }
 
@@ -245,9 +247,10 @@ __device__ __forceinline__ bool issue_pv(uint64_t* bars, uint32_t tmem, uint32_t
   return true;
 }
 
-template <int DP, bool WIN>
+template <int DP, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<DP>;
+  constexpr bool WIN = MODE == kModeWindow;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {                       // layout needs 1024-byte alignment
     if (threadIdx.x == 0) atomicCAS(p.status, 0, DT_ERR_UNSUPPORTED);
@@ -313,9 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
-        if (!item_has_compute<WIN>(G, qt, cm)) continue;
+        if (!item_has_compute<MODE>(G, qt, cm)) continue;
         if (is_k) {
-          const QTile t = query_tile<WIN>(G, qt);
+          const QTile t = query_tile<MODE>(G, qt);
           if (nq > 0 && !mbar_wait(&bars[C::bQEmpty], (nq - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
             goto tma_done;
           mbar_arrive_expect_tx(&bars[C::bQFull], C::kTileBytes);
@@ -328,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         for (int j = 0; j < G.P; ++j) {
           const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
-          const KeySet ks = key_set<WIN>(G, qt, seg);
+          const KeySet ks = key_set<MODE>(G, qt, seg);
           const int nt = ks.ntiles();
           const int toff = nt > 0 ? tile_rotation(nt, idx, seg) : 0;
           for (int i = 0; i < nt; ++i, ++g) {
@@ -336,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             if (g >= (uint32_t)C::kStages &&
                 !mbar_wait(&empty[st], ((g / C::kStages) - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
               goto tma_done;
-            const int row0 = ks.base + visit_tile(ks, nt, toff, i) * kTile;
+            const int row0 = ks.row0(visit_tile(ks, nt, toff, i));
             uint8_t* dst = ring + st * C::kTileBytes;
             DT_TR(is_k ? 8 : 9, g);
             mbar_arrive_expect_tx(&full[st], C::kTileBytes);
@@ -371,14 +374,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
-        if (!item_has_compute<WIN>(G, qt, cm)) continue;
+        if (!item_has_compute<MODE>(G, qt, cm)) continue;
         if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
         ++nq;
         tc_fence_after();
         for (int j = 0; j < G.P && ok; ++j) {
           const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
-          const int nt = key_set<WIN>(G, qt, seg).ntiles();
+          const int nt = key_set<MODE>(G, qt, seg).ntiles();
           if (nt == 0) continue;
           for (int i = 0; i < nt; ++i, ++g) {
             const int st = g % C::kStages;
@@ -443,11 +446,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
-        if (!item_has_compute<WIN>(G, qt, cm)) continue;
+        if (!item_has_compute<MODE>(G, qt, cm)) continue;
         for (int j = 0; j < G.P && ok; ++j) {
           const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
-          const int nt = key_set<WIN>(G, qt, seg).ntiles();
+          const int nt = key_set<MODE>(G, qt, seg).ntiles();
           if (nt == 0) continue;
           for (int i = 0; i < nt && ok; ++i, ++g)
             ok = issue_pv<DP>(bars, tmem, aV, g, cseg, i == 0, i == nt - 1, WIN && seg == 0, abort_flag, p.status,
@@ -478,14 +481,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const int qt = idx - (idx / G.nqt) * G.nqt;
       const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
       const int rot = seg_rotation<WIN>(G, idx);
-      if (!item_has_compute<WIN>(G, qt, cm)) continue;
-      const QTile t = query_tile<WIN>(G, qt);
+      if (!item_has_compute<MODE>(G, qt, cm)) continue;
+      const QTile t = query_tile<MODE>(G, qt);
       const int qa = t.q0 + ra, qb = t.q0 + rb;
       const int q1 = t.q0 + t.rows - 1;
       for (int j = 0; j < G.P; ++j) {
         const int seg = visit_seg<WIN>(G, rot, j);
         if (!is_compute(cm, seg)) continue;
-        const KeySet ks = key_set<WIN>(G, qt, seg);
+        const KeySet ks = key_set<MODE>(G, qt, seg);
         const int nt = ks.ntiles();
         if (nt == 0) continue;
         const int toff = tile_rotation(nt, idx, seg);
@@ -501,8 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           if (warp == 7) DT_TR(14, g);
           tc_fence_after();
           const int tile = visit_tile(ks, nt, toff, i);
-          const int k0 = ks.base + tile * kTile;
-          const int kvalid = imin(kTile, ks.kend - k0);
+          const int k0 = ks.row0(tile);
+          const int kvalid = imin(kTile, ks.rowend(tile) - k0);
           const uint32_t sc = tmem + lane_base + C::kColS + sb * 128;
           uint32_t sr[64];
           tmem_ld_16x256b_x8(sc, sr);
@@ -665,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
       const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
       const int rot = seg_rotation<WIN>(G, idx);
-      const QTile t = query_tile<WIN>(G, qt);
+      const QTile t = query_tile<MODE>(G, qt);
       const int qrow = t.q0 + r;
       const bool valid = r < t.rows;
       float m_tot = kNegInf, l_tot = 0.f;
@@ -685,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         for (; jr < G.P; ++jr) {
           const int seg = visit_seg<WIN>(G, rot, jr);
           if (is_compute(cm, seg)) continue;
-          n_skip += counted_blocks<WIN>(G, qt, seg);   // same in every lane; thread 0 reports
+          n_skip += counted_blocks<MODE>(G, qt, seg);   // same in every lane; thread 0 reports
           ++n_read;
           if (WIN) { use_r = true; ++merged; continue; }   // complement reused: add R at the end
           const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
@@ -730,9 +733,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       for (int j = 0; j < G.P; ++j) {
         const int seg = visit_seg<WIN>(G, rot, j);
         if (!is_compute(cm, seg)) continue;
-        const int nt = key_set<WIN>(G, qt, seg).ntiles();
+        const int nt = key_set<MODE>(G, qt, seg).ntiles();
         const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
-        n_comp += counted_blocks<WIN>(G, qt, seg);
+        n_comp += counted_blocks<MODE>(G, qt, seg);
         ++n_fresh;
         if (nt == 0) {             // empty key set: the identity state
           if (!WIN && valid) {
@@ -839,17 +842,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   }
 }
 
-template <int DP, bool WIN>
+template <int DP, int MODE>
 int launch_dp(const AttnParams& kp, int grid, cudaStream_t stream) {
   using C = Cfg<DP>;
   static bool attr_set = false;   // per-process; the attribute is per device function
   if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_partial_fused_kernel<DP, WIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(attn_partial_fused_kernel<DP, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmem) != cudaSuccess)
       return DT_ERR_CUDA;
     attr_set = true;
   }
-  attn_partial_fused_kernel<DP, WIN><<<grid, kThreads, C::kSmem, stream>>>(kp);
+  attn_partial_fused_kernel<DP, MODE><<<grid, kThreads, C::kSmem, stream>>>(kp);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
 }
 
@@ -870,12 +873,18 @@ int attn_fused_smem_bytes(int dp) {
   return -1;
 }
 
+template <int DP>
+int launch_mode(const AttnParams& kp, int grid, cudaStream_t stream) {
+  if (kp.window > 0) return launch_dp<DP, kModeWindow>(kp, grid, stream);
+  if (kp.geom.grp > 0) return launch_dp<DP, kModeGrouped>(kp, grid, stream);
+  return launch_dp<DP, kModePartition>(kp, grid, stream);
+}
+
 int launch_attn_fused(const AttnParams& kp, int dp, int grid, cudaStream_t stream) {
   switch (dp) {
-    case 64: return kp.window > 0 ? launch_dp<64, true>(kp, grid, stream) : launch_dp<64, false>(kp, grid, stream);
-    case 80: return kp.window > 0 ? launch_dp<80, true>(kp, grid, stream) : launch_dp<80, false>(kp, grid, stream);
-    case 128:
-      return kp.window > 0 ? launch_dp<128, true>(kp, grid, stream) : launch_dp<128, false>(kp, grid, stream);
+    case 64: return launch_mode<64>(kp, grid, stream);
+    case 80: return launch_mode<80>(kp, grid, stream);
+    case 128: return launch_mode<128>(kp, grid, stream);
   }
   return DT_ERR_UNSUPPORTED;
 }

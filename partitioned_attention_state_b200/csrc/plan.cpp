@@ -6,7 +6,9 @@
 // distant ones; spatial locality (Fig. 5a) ranks partitions by distance; anchor
 // steps compute everything.  "DiTFastAttn: Attention Compression for Diffusion
 // Transformer Models" (Approach): window attention with a cached residual is
-// expressed as two key sets per query tile (window, complement).
+// expressed as two key sets per query tile (window, complement).  State
+// grouping (grouping of spatially adjacent states) makes a key set a group of
+// partitions; the proximity rule then ranks groups.
 #include <cstring>
 #include <vector>
 
@@ -19,19 +21,46 @@ bool params_ok(const dt_plan_params* p) {
   if (!p) return false;
   if (p->H < 0 || p->S < 0 || p->D < 1 || p->step < 1) return false;
   if (p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW) return false;
+  if (p->group < 0) return false;
   if (p->mode == DT_MODE_WINDOW) {
-    if (p->window < 1) return false;
+    if (p->window < 1 || p->group != 0) return false;
   } else {
     if (p->P < 1) return false;
-    if (p->mode == DT_MODE_PROXIMITY && (p->reuse_per_row < 0 || p->reuse_per_row > p->P - 1))
-      return false;
+    const int rmax = p->group > 0 ? dt::ceil_div(p->P, p->group) : p->P - 1;
+    if (p->mode == DT_MODE_PROXIMITY && (p->reuse_per_row < 0 || p->reuse_per_row > rmax)) return false;
   }
   return true;
 }
 
 dt::Geom geom_of(const dt_plan_params* p) {
   return p->mode == DT_MODE_WINDOW ? dt::make_geom(p->H, p->S, p->D, 1, p->window)
-                                   : dt::make_geom(p->H, p->S, p->D, p->P, 0);
+                                   : dt::make_geom(p->H, p->S, p->D, p->P, 0, p->group);
+}
+
+// Grouped proximity row of a query in partition q (1 + m entries): set 0 (the
+// local partition) is computed; the r groups farthest from q's group are
+// reused, equal distances in increasing index order.
+void group_proximity_row(int q, int m, int g, int r, uint8_t* row) {
+  for (int k = 0; k <= m; ++k) row[k] = DT_PLAN_COMPUTE;
+  const int lg = q / g;
+  int taken = 0;
+  for (int dist = m - 1; dist >= 0 && taken < r; --dist) {
+    int cand[2] = {lg - dist, lg + dist};
+    for (int c = 0; c < (dist == 0 ? 1 : 2) && taken < r; ++c) {
+      if (cand[c] >= 0 && cand[c] < m) { row[1 + cand[c]] = DT_PLAN_REUSE; ++taken; }
+    }
+  }
+}
+
+// Keys of key set k of query tile qt (partition modes).
+int64_t set_keys(const dt::Geom& g, int qt, int k) {
+  if (g.grp == 0) return dt::part_end(g, k) - dt::part_begin(g, k);
+  const int q = dt::query_tile<0>(g, qt).part;
+  if (k == 0) return dt::part_end(g, q) - dt::part_begin(g, q);
+  const int a = (k - 1) * g.grp, b = dt::imin(k * g.grp, g.parts);
+  int64_t n = dt::part_end(g, b - 1) - dt::part_begin(g, a);
+  if (a <= q && q < b) n -= dt::part_end(g, q) - dt::part_begin(g, q);
+  return n;
 }
 
 // Proximity row of query partition q: reuse the r partitions farthest from q,
@@ -94,6 +123,7 @@ extern "C" int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_pl
         break;
       case DT_MODE_PROXIMITY:
         if (anchor) { for (int k = 0; k < nseg; ++k) row[k] = DT_PLAN_COMPUTE; }
+        else if (g.grp > 0) group_proximity_row(dt::query_tile(g, qt).part, nseg - 1, g.grp, p->reuse_per_row, row);
         else proximity_row(dt::query_tile(g, qt).part, nseg, p->reuse_per_row, row);
         break;
       case DT_MODE_ALL_REUSE:
@@ -145,8 +175,8 @@ extern "C" int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_pl
       }
     } else {
       for (int k = 0; k < nseg; ++k) {
-        int len = dt::part_end(g, k) - dt::part_begin(g, k);
-        int64_t nb = H * dt::ceil_div(len, dt::kTile);
+        const int64_t len = set_keys(g, qt, k);
+        int64_t nb = H * dt::counted_blocks(g, qt, k);
         if (row[k] == DT_PLAN_COMPUTE) {
           cb += nb;
           fl += 4 * H * D * (int64_t)t.rows * len;

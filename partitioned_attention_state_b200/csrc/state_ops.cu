@@ -1,5 +1,6 @@
 // state_ops.cu -- HBM-bound state kernels of libdt: N-way state composition,
-// plan-driven cache scatter, and the window residual (make / apply).
+// plan-driven cache scatter, in-place regrouping of cached group states, and
+// the window residual (make / apply).
 //
 // All three stream rows of D fp32 values with 16-byte vector accesses over a
 // flat index, so consecutive threads touch consecutive 16-byte words (fully
@@ -96,6 +97,53 @@ __global__ void __launch_bounds__(kBlock) window_residual_kernel(int op, int64_t
   }
 }
 
+// "DiTango", Dynamic Group State Compose: cached group states are merged
+// `factor` at a time into coarser groups (Eq. 4 composition), in place.  One
+// warp owns a (head, row) and walks the new groups in increasing order; new
+// group i reads old slots 1 + factor*i .. (all at or after slot 1 + i) and
+// writes slot 1 + i, which only an already finished group read.  Inside a
+// group every lane reads all inputs (the LSEs are shared by the whole row)
+// before any lane writes, so the write of slot 1 + i cannot race a read of it.
+__global__ void __launch_bounds__(kBlock) group_compose_kernel(int m, int factor, int64_t rows, int D,
+                                                               float* __restrict__ cO, float* __restrict__ cL) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (kBlock / 32);
+  const int m2 = (m + factor - 1) / factor;
+  const int d4n = D / 4;
+  for (int64_t row = blockIdx.x * (int64_t)(kBlock / 32) + (threadIdx.x >> 5); row < rows; row += warps) {
+    for (int i = 0; i < m2; ++i) {
+      const int j0 = 1 + factor * i, n = min(factor, m - factor * i);
+      float M = kNegInf;
+      for (int k = 0; k < n; ++k) M = fmaxf(M, cL[(int64_t)(j0 + k) * rows + row]);
+      float Lr = kNegInf, tot = 0.f;
+      if (M > kNegInf) {
+        for (int k = 0; k < n; ++k) tot += expf(cL[(int64_t)(j0 + k) * rows + row] - M);
+        Lr = M + logf(tot);
+      }
+      float w[8];                               // factor <= 8 (checked on the host)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        w[k] = (k < n && M > kNegInf) ? expf(cL[(int64_t)(j0 + k) * rows + row] - Lr) : 0.f;
+      // each lane composes its own columns: it reads them all before writing
+      for (int c4 = lane; c4 < d4n; c4 += 32) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < n; ++k) {
+          if (w[k] == 0.f) continue;
+          const float4 v = reinterpret_cast<const float4*>(cO + ((int64_t)(j0 + k) * rows + row) * D)[c4];
+          acc.x = fmaf(w[k], v.x, acc.x);
+          acc.y = fmaf(w[k], v.y, acc.y);
+          acc.z = fmaf(w[k], v.z, acc.z);
+          acc.w = fmaf(w[k], v.w, acc.w);
+        }
+        reinterpret_cast<float4*>(cO + ((int64_t)(1 + i) * rows + row) * D)[c4] = acc;
+      }
+      __syncwarp();                             // every lane has read this group's LSEs
+      if (lane == 0) cL[(int64_t)(1 + i) * rows + row] = Lr;
+      __syncwarp();
+    }
+  }
+}
+
 int grid_for(int64_t work, int sms) {
   int64_t blocks = (work + kBlock - 1) / kBlock;
   int64_t cap = (int64_t)sms * 8;           // 8 resident 256-thread blocks per SM
@@ -117,6 +165,12 @@ int launch_cache_update(const Geom& G, const uint8_t* plan, const float* fO, con
                         int sms, cudaStream_t st) {
   const int64_t work = (int64_t)G.P * G.H * G.S * (G.D / 4);
   cache_update_kernel<<<grid_for(work, sms), kBlock, 0, st>>>(G, plan, fO, fL, cO, cL);
+  return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+}
+
+int launch_group_compose(int m, int factor, int H, int S, int D, float* cO, float* cL, int sms, cudaStream_t st) {
+  const int64_t rows = (int64_t)H * S;
+  group_compose_kernel<<<grid_for(rows * 32, sms), kBlock, 0, st>>>(m, factor, rows, D, cO, cL);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
 }
 

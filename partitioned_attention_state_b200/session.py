@@ -16,8 +16,8 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused, dt_attn_partial_fused_heads, dt_plan_build,
-               dt_plan_geometry, DtError, params)
+from . import (DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused, dt_attn_partial_fused_heads, dt_group_compose,
+               dt_plan_build, dt_plan_geometry, DtError, params)
 
 
 def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
@@ -28,12 +28,16 @@ def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
 
 class Session:
     def __init__(self, H: int, S: int, D: int, P: int = 1, mode: int = DT_MODE_PROXIMITY, reuse_per_row: int = 0,
-                 window: int = 0, device: str = "cuda", cache: bool = True):
+                 window: int = 0, device: str = "cuda", cache: bool = True, group: int = 0):
+        """group: 0 = one key set (and cache slot) per partition; g >= 1 =
+        state grouping (the local partition, then groups of g adjacent
+        partitions); reuse_per_row then counts groups."""
         self.H, self.S, self.D, self.P = H, S, D, P
         self.mode, self.r, self.window = mode, reuse_per_row, window
+        self.group = group
         self.device = torch.device(device)
         win = mode == DT_MODE_WINDOW
-        p = params(H, S, D, P if not win else 1, mode, reuse_per_row, window, 1)
+        p = params(H, S, D, P if not win else 1, mode, reuse_per_row, window, 1, group)
         self.nqt, self.nseg = dt_plan_geometry(p)
         dev = self.device
         self.Q = torch.empty((H, S, D), dtype=torch.bfloat16, device=dev)
@@ -45,21 +49,44 @@ class Session:
             self.cache_O = self.cache_L = None
             self.R = torch.zeros((H, S, D), dtype=torch.float32, device=dev)
         else:
-            self.cache_O = torch.zeros((P, H, S, D), dtype=torch.float32, device=dev) if cache else None
-            self.cache_L = torch.full((P, H, S), float("-inf"), dtype=torch.float32, device=dev) if cache else None
+            ns = self.nseg
+            self.cache_O = torch.zeros((ns, H, S, D), dtype=torch.float32, device=dev) if cache else None
+            self.cache_L = torch.full((ns, H, S), float("-inf"), dtype=torch.float32, device=dev) if cache else None
             self.R = None
-        self.d_plan = torch.zeros((max(self.nqt, 1), self.nseg), dtype=torch.uint8, device=dev)
+        self._plan_buffers()
+        self.counters = torch.zeros(4, dtype=torch.int64, device=dev)
+        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
+        self.stamps = np.full((self.nqt, self.nseg), -1, dtype=np.int32)
+        self.last_counts = None
+        self.last_plan = None
+
+    def _plan_buffers(self) -> None:
+        self.d_plan = torch.zeros((max(self.nqt, 1), self.nseg), dtype=torch.uint8, device=self.device)
         # two pinned host plan buffers: the plan of step t is built while the
         # upload of step t-1 may still be in flight
         self._pinned = [torch.zeros((max(self.nqt, 1), self.nseg), dtype=torch.uint8, pin_memory=True)
                         for _ in range(2)]
         self._uploaded = [None, None]
         self._turn = 0
-        self.counters = torch.zeros(4, dtype=torch.int64, device=dev)
-        self.status = torch.zeros(4, dtype=torch.int32, device=dev)
-        self.stamps = np.full((self.nqt, self.nseg), -1, dtype=np.int32)
-        self.last_counts = None
-        self.last_plan = None
+
+    def compose_groups(self, factor: int = 2, shrink: bool = False) -> None:
+        """Dynamic Group State Compose: regroup the cached group states into
+        groups `factor` times coarser (in place on the device, stamps on the
+        host); later steps plan on the coarser groups.  ``shrink`` moves the
+        cache into buffers of the new size (a copy) to give memory back."""
+        if self.group < 1 or self.cache_O is None:
+            raise ValueError("compose_groups needs a grouped session with a cache")
+        p = params(self.H, self.S, self.D, self.P, self.mode, self.r, 0, 1, self.group)
+        for ev in self._uploaded:
+            if ev is not None:
+                ev.synchronize()
+        self.stamps = dt_group_compose(p, factor, self.stamps, self.cache_O, self.cache_L, self.status).copy()
+        self.group *= factor
+        self.nseg = self.stamps.shape[1]
+        if shrink:
+            self.cache_O = self.cache_O[: self.nseg].clone()
+            self.cache_L = self.cache_L[: self.nseg].clone()
+        self._plan_buffers()
 
     # -------------------------------------------------------------- inputs
     def set_inputs(self, q, k, v) -> None:
@@ -74,7 +101,8 @@ class Session:
     def plan(self, step: int, mode: Optional[int] = None, explicit: Optional[np.ndarray] = None):
         mode = self.mode if mode is None else mode
         win = mode == DT_MODE_WINDOW
-        p = params(self.H, self.S, self.D, 1 if win else self.P, mode, self.r, self.window, step)
+        p = params(self.H, self.S, self.D, 1 if win else self.P, mode, self.r, self.window, step,
+                   0 if win else self.group)
         plan, counts = dt_plan_build(p, self.stamps, explicit)
         return p, plan, counts
 

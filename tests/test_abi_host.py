@@ -38,12 +38,12 @@ def test_status_strings():
     assert "unknown" in dt.dt_status_string(12345)
 
 
-def run_both(mode, H, S, D, P, step, r=0, window=0, stamps=None, explicit=None):
-    p = dt.params(H, S, D, P, mode, r, window, step)
+def run_both(mode, H, S, D, P, step, r=0, window=0, stamps=None, explicit=None, group=0):
+    p = dt.params(H, S, D, P, mode, r, window, step, group)
     st_c = None if stamps is None else stamps.copy()
     plan_c, counts_c = dt.dt_plan_build(p, st_c, explicit)
     plan_o, counts_o, st_o = orc.build_plan(mode, H, S, D, P if mode != orc.MODE_WINDOW else 1, step, r=r,
-                                            window=window, stamps=stamps, explicit=explicit)
+                                            window=window, stamps=stamps, explicit=explicit, group=group)
     np.testing.assert_array_equal(plan_c, plan_o)
     assert counts_c == counts_o
     if st_c is not None:
@@ -175,3 +175,74 @@ def test_head_range_validated_on_the_host():
     # a valid range still needs its buffers
     assert lib.dt_attn_partial_fused_heads(ctypes.byref(p), 1, 2, *([None] * 11), None) == dt.DT_ERR_INVALID
     assert lib.dt_attn_partial_fused_heads(None, 0, 1, *([None] * 11), None) == dt.DT_ERR_INVALID
+
+
+@pytest.mark.parametrize("S,P,g,r", [(32760, 16, 4, 2), (16384, 16, 4, 1), (1024, 8, 2, 2), (1000, 3, 2, 1),
+                                     (5, 4, 3, 1), (4097, 7, 3, 2), (300, 5, 1, 4), (2600, 64, 8, 3),
+                                     (640, 4, 4, 1), (130, 2, 2, 1)])
+def test_grouped_plan_matches_oracle(S, P, g, r):
+    """State grouping: geometry, plans, counts and stamps of the C builder
+    equal the oracle's, bit for bit, through a schedule of every mode."""
+    H, D = 3, 64
+    p = dt.params(H, S, D, P, dt.DT_MODE_PROXIMITY, r, 0, 1, g)
+    nqt, nseg = dt.dt_plan_geometry(p)
+    assert nqt == len(orc.query_tiles(S, P)) and nseg == 1 + -(-P // g)
+    st = np.full((nqt, nseg), -1, np.int32)
+    _, _, st = run_both(orc.MODE_PROXIMITY, H, S, D, P, 1, r=r, stamps=st, group=g)
+    _, c2, st = run_both(orc.MODE_PROXIMITY, H, S, D, P, 2, r=r, stamps=st, group=g)
+    run_both(orc.MODE_ALL_REUSE, H, S, D, P, 3, stamps=st, group=g)
+    ex = (np.arange(nqt * nseg).reshape(nqt, nseg) % 3 == 0).astype(np.uint8)
+    run_both(orc.MODE_EXPLICIT, H, S, D, P, 3, stamps=st, explicit=ex, group=g)
+    _, call, _ = run_both(orc.MODE_ALL_COMPUTE, H, S, D, P, 4, group=g)
+    # grouping only regroups the blocks: the anchor computes every block once
+    _, cflat = dt.dt_plan_build(dt.params(H, S, D, P, dt.DT_MODE_ALL_COMPUTE, 0, 0, 1), None)
+    assert call == cflat
+
+
+def test_grouped_params_validated():
+    import ctypes
+    lib = dt.load()
+    nqt, nseg = ctypes.c_int32(), ctypes.c_int32()
+    bad = [dt.params(1, 1024, 64, 16, dt.DT_MODE_PROXIMITY, 5, 0, 1, 4),   # r > m = 4
+           dt.params(1, 1024, 64, 16, dt.DT_MODE_PROXIMITY, 1, 0, 1, -1),
+           dt.params(1, 1024, 64, 1, dt.DT_MODE_WINDOW, 0, 64, 1, 2)]      # grouping is for partitions
+    for p in bad:
+        assert lib.dt_plan_geometry(ctypes.byref(p), ctypes.byref(nqt), ctypes.byref(nseg)) == dt.DT_ERR_INVALID
+    ok = dt.params(1, 1024, 64, 16, dt.DT_MODE_PROXIMITY, 4, 0, 1, 4)        # r = m: the local group too
+    assert lib.dt_plan_geometry(ctypes.byref(ok), ctypes.byref(nqt), ctypes.byref(nseg)) == dt.DT_OK
+    # the fused kernel keeps a plan row as a 64-bit mask: at most 64 key sets
+    p = dt.params(1, 128 * 130, 64, 130, dt.DT_MODE_ALL_COMPUTE, 0, 0, 1, 2)   # 1 + 65 sets
+    assert lib.dt_attn_partial_fused(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_UNSUPPORTED
+    p.group = 3                                                             # 1 + 44 sets
+    assert lib.dt_attn_partial_fused(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_INVALID
+
+
+@pytest.mark.parametrize("P,g,f", [(16, 1, 2), (16, 2, 2), (16, 4, 2), (8, 1, 3), (5, 1, 2), (7, 2, 4), (16, 1, 8)])
+def test_group_compose_stamps_match_oracle(P, g, f):
+    """Host half of Dynamic Group State Compose (H = 0: no device work): the
+    stamps of the coarse layout equal the oracle's, and the coarse layout's
+    geometry is that of group size g * f."""
+    S = 128 * P
+    p = dt.params(0, S, 64, P, dt.DT_MODE_PROXIMITY, 0, 0, 1, g)
+    nqt, nseg = dt.dt_plan_geometry(p)
+    rng = np.random.default_rng(P * 100 + g * 10 + f)
+    st = rng.integers(-1, 9, size=(nqt, nseg)).astype(np.int32)
+    _, want = orc.compose_groups(orc.StateCache(), st, P, g, f, [], np.zeros(0, int), S, 64)
+    got = dt.dt_group_compose(p, f, st.copy(), None, None, stream=0)
+    np.testing.assert_array_equal(got, want)
+    assert got.shape[1] == dt.dt_plan_geometry(dt.params(0, S, 64, P, dt.DT_MODE_PROXIMITY, 0, 0, 1, g * f))[1]
+
+
+def test_group_compose_validated():
+    import ctypes
+    lib = dt.load()
+    p = dt.params(2, 1024, 64, 8, dt.DT_MODE_PROXIMITY, 0, 0, 1, 2)
+    assert lib.dt_group_compose(ctypes.byref(p), 1, None, None, None, None, None) == dt.DT_ERR_INVALID  # factor
+    assert lib.dt_group_compose(ctypes.byref(p), 2, None, None, None, None, None) == dt.DT_ERR_INVALID  # no cache
+    p.group = 0
+    assert lib.dt_group_compose(ctypes.byref(p), 2, None, None, None, None, None) == dt.DT_ERR_INVALID  # ungrouped
+    p.group, p.D = 2, 66
+    assert lib.dt_group_compose(ctypes.byref(p), 2, None, None, None, None, None) == dt.DT_ERR_INVALID
+    p.D = 64
+    assert lib.dt_group_compose(ctypes.byref(p), 2, None, 16 * 1024 + 4, 16 * 1024, None, None) == \
+        dt.DT_ERR_UNSUPPORTED

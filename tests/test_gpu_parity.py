@@ -30,10 +30,14 @@ def _gpu():
 
 
 def run_partition_schedule(H, S, D, P, schedule, inputs, heads=None, rows=None, check_untouched=False,
-                           output_scaled=False):
-    """schedule: list of (step, mode, r, explicit); inputs: callable -> (q,k,v) bits."""
-    sess = Session(H, S, D, P, mode=dt.DT_MODE_PROXIMITY)
-    cache = orc.StateCache()
+                           output_scaled=False, group=0, sess=None, cache=None):
+    """schedule: list of (step, mode, r, explicit); inputs: callable -> (q,k,v) bits.
+    group > 0: grouped key sets (one cache slot per group).  A session and
+    oracle cache may be passed in to continue an earlier schedule."""
+    if sess is None:
+        sess = Session(H, S, D, P, mode=dt.DT_MODE_PROXIMITY, group=group)
+        cache = orc.StateCache()
+    group = sess.group
     hs = list(range(H)) if heads is None else list(heads)
     rs = np.arange(S) if rows is None else np.asarray(rows)
     for step, mode, r, explicit in schedule:
@@ -52,7 +56,7 @@ def run_partition_schedule(H, S, D, P, schedule, inputs, heads=None, rows=None, 
         assert int(c[0]) == counts["computed_blocks"] and int(c[1]) == counts["skipped_blocks"]
         assert int(c[2]) == H * int((plan == 1).sum()) and int(c[3]) == H * int((plan == 0).sum())
         Q, K, V = (orc.widen_bf16(x[hs]) for x in (q, k, v))
-        O_ref, L_ref, fresh = orc.partition_step(Q, K, V, plan, S, P, cache, rows=rs)
+        O_ref, L_ref, fresh = orc.partition_step(Q, K, V, plan, S, P, cache, rows=rs, group=group)
         O_gpu = to_np(sess.O[hs][:, rs])
         L_gpu = to_np(sess.L[hs][:, rs])
         check_out(O_gpu, O_ref, f"O step {step}", output_scaled=output_scaled)
@@ -68,11 +72,11 @@ def run_partition_schedule(H, S, D, P, schedule, inputs, heads=None, rows=None, 
         if before is not None:
             tiles = orc.query_tiles(S, P)
             for t, (_, q0, q1) in enumerate(tiles):
-                for kk in range(P):
+                for kk in range(sess.nseg):
                     if plan[t, kk] == orc.REUSE:
                         assert torch.equal(before[0][kk, :, q0:q1], co[kk, :, q0:q1])
                         assert torch.equal(before[1][kk, :, q0:q1], cl[kk, :, q0:q1])
-    return sess
+    return sess, cache
 
 
 def proximity_schedule(steps, r):
@@ -162,7 +166,7 @@ def test_all_reuse_reproduces_previous_output_and_explicit_plan():
     nqt = len(orc.query_tiles(S, P))
     ex = (np.arange(nqt * P).reshape(nqt, P) % 2).astype(np.uint8)
     sched.append((3, dt.DT_MODE_EXPLICIT, 0, ex))
-    sess = run_partition_schedule(H, S, D, P, sched, lambda: (q, k, v))
+    sess, _ = run_partition_schedule(H, S, D, P, sched, lambda: (q, k, v))
     # with unchanged inputs every plan gives full attention
     full, lf = orc.attention_state(orc.widen_bf16(q[1]), orc.widen_bf16(k[1]), orc.widen_bf16(v[1]),
                                    orc.softmax_scale(D))
@@ -308,3 +312,63 @@ def test_host_step_window_mode_matches_whole_step():
         assert torch.equal(a.O.view(torch.int16).cpu(), ho)
         assert torch.equal(a.L.cpu(), hl)
         assert torch.equal(a.R, b.R)
+
+
+
+# ------------------------------------------------------------ state grouping
+
+@pytest.mark.parametrize("H,S,D,P,g,rs", [
+    (16, 1024, 72, 8, 2, (1, 2, 3)),     # DiT-XL/2-like geometry, groups of 2
+    (2, 1024, 64, 4, 2, (1, 2)),         # the Fig. 6 layout (CP = 4, groups of 2)
+    (2, 2048, 128, 16, 4, (2, 1, 3)),    # the video grouping on a short sequence
+    (1, 2600, 64, 64, 8, (3, 7)),        # 1 + 8 key sets, 41-row partitions (one short tile each)
+    (2, 1800, 72, 12, 5, (1, 2)),        # last group short, 150-row partitions (ragged tiles)
+    (1, 1000, 128, 7, 3, (2,)),          # P not a multiple of g, ragged last partition
+    (2, 1024, 72, 8, 1, (3, 7)),         # groups of one: 1 + P key sets, the local group empty
+])
+def test_grouped_schedule_parity(H, S, D, P, g, rs):
+    sched = [(1, dt.DT_MODE_PROXIMITY, rs[0], None)] + \
+            [(t + 2, dt.DT_MODE_PROXIMITY, r, None) for t, r in enumerate(rs)]
+    run_partition_schedule(H, S, D, P, sched, stream_of(H, S, D, 0.05, seed=S + g), check_untouched=True, group=g)
+
+
+def test_grouped_video_full_size_sampled_rows():
+    """The video workload with groups of 4 partitions (1 + 4 key sets) in the
+    benchmark's launch configuration: anchor, then 2 of 4 groups reused."""
+    w = wl.WORKLOADS[3]
+    sched = [(1, dt.DT_MODE_PROXIMITY, 2, None), (2, dt.DT_MODE_PROXIMITY, 2, None),
+             (3, dt.DT_MODE_PROXIMITY, 3, None)]
+    run_partition_schedule(w.H, w.S, w.D, w.P, sched, wl.stream_for(w).next_step, heads=[0, 39],
+                           rows=sample_rows(w.S, w.P, n_extra=24), group=4)
+
+
+@pytest.mark.parametrize("P,g,f", [(8, 1, 2), (16, 2, 2), (12, 1, 3), (7, 2, 4)])
+def test_group_compose_matches_oracle(P, g, f):
+    """Dynamic Group State Compose on the GPU: the regrouped cache equals the
+    oracle's N-way composition of the GPU's own cached states (fp32 rounding
+    only), the stamps equal the oracle's, and later steps on the coarse
+    layout match the oracle run through the same regrouping."""
+    H, S, D = 2, 128 * P + 40, 64
+    s = stream_of(H, S, D, 0.05, seed=P * 10 + g)
+    sess, cache = run_partition_schedule(H, S, D, P, [(1, dt.DT_MODE_PROXIMITY, 1, None),
+                                                      (2, dt.DT_MODE_PROXIMITY, 1, None)], s, group=g)
+    m = -(-P // g)
+    before_O = to_np(sess.cache_O[: 1 + m])
+    before_L = to_np(sess.cache_L[: 1 + m])
+    st_before = sess.stamps.copy()
+    sess.compose_groups(f)
+    sess.check()
+    m2 = -(-m // f)
+    assert sess.group == g * f and sess.nseg == 1 + m2
+    new_cache, st_want = orc.compose_groups(cache, st_before, P, g, f, list(range(H)), np.arange(S), S, D)
+    np.testing.assert_array_equal(sess.stamps, st_want)
+    np.testing.assert_array_equal(to_np(sess.cache_O[0]), before_O[0])
+    for i in range(m2):
+        js = range(f * i, min(f * i + f, m))
+        want_o, want_l = orc.compose_n([(before_O[1 + j].reshape(-1, D), before_L[1 + j].reshape(-1)) for j in js])
+        got_o = to_np(sess.cache_O[1 + i]).reshape(-1, D)
+        got_l = to_np(sess.cache_L[1 + i]).reshape(-1)
+        np.testing.assert_allclose(got_o, want_o, rtol=2e-5, atol=2e-6)
+        np.testing.assert_allclose(got_l, want_l, rtol=0, atol=2e-5)
+    run_partition_schedule(H, S, D, P, [(3, dt.DT_MODE_PROXIMITY, 1, None), (4, dt.DT_MODE_ALL_REUSE, 0, None)], s,
+                           sess=sess, cache=new_cache)
