@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--eager", action="store_true",
                     help="launch every timed step through the host path instead of replaying a captured CUDA graph")
     ap.add_argument("--heads", type=int, default=None, help="override H (smaller profiling captures)")
+    ap.add_argument("--group", type=int, default=0,
+                    help="state grouping: groups of G adjacent partitions, --reuse then counts groups")
+    ap.add_argument("--no-grouped", action="store_true", help="skip the grouped-cache and compose measurements")
     return ap.parse_args()
 
 
@@ -168,7 +171,7 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- oracle leg
 
-def oracle_sample(w, r, budget_s=12.0, heads=(0,), inputs=None):
+def oracle_sample(w, r, budget_s=12.0, heads=(0,), inputs=None, group=0):
     """Time the CPU oracle on a bounded sample of one reuse step: whole query
     tiles (all their computed partial states, cached-state merges and the
     cache update) of one head, until about budget_s seconds of work."""
@@ -186,8 +189,8 @@ def oracle_sample(w, r, budget_s=12.0, heads=(0,), inputs=None):
     hs = list(heads)
     tiles = orc.query_tiles(w.S, w.P)
     nqt = len(tiles)
-    plan1, _, st = orc.build_plan(orc.MODE_PROXIMITY, w.H, w.S, w.D, w.P, 1, r=r)
-    plan2, counts, _ = orc.build_plan(orc.MODE_PROXIMITY, w.H, w.S, w.D, w.P, 2, r=r, stamps=st)
+    plan1, _, st = orc.build_plan(orc.MODE_PROXIMITY, w.H, w.S, w.D, w.P, 1, r=r, group=group)
+    plan2, counts, _ = orc.build_plan(orc.MODE_PROXIMITY, w.H, w.S, w.D, w.P, 2, r=r, stamps=st, group=group)
     Q1, K1, V1 = (orc.widen_bf16(x[hs]) for x in (q1, k1, v1))
     Q2, K2, V2 = (orc.widen_bf16(x[hs]) for x in (q2, k2, v2))
     parts = orc.partitions(w.S, w.P)
@@ -200,22 +203,26 @@ def oracle_sample(w, r, budget_s=12.0, heads=(0,), inputs=None):
         _, q0, qe = tiles[t]
         rows = np.arange(q0, qe)
         cache = orc.StateCache()
-        orc.partition_step(Q1, K1, V1, plan1, w.S, w.P, cache, rows=rows)     # anchor fills the cache (untimed)
+        orc.partition_step(Q1, K1, V1, plan1, w.S, w.P, cache, rows=rows, group=group)   # anchor (untimed)
         t0 = time.perf_counter()
-        orc.partition_step(Q2, K2, V2, plan2, w.S, w.P, cache, rows=rows)
+        orc.partition_step(Q2, K2, V2, plan2, w.S, w.P, cache, rows=rows, group=group)
         elapsed += time.perf_counter() - t0
-        flops += sum(4 * w.D * len(hs) * (qe - q0) * (b - a) for k, (a, b) in enumerate(parts) if plan2[t, k])
+        sets = orc.key_sets_of_tile(tiles[t][0], w.P, group)
+        flops += sum(4 * w.D * len(hs) * (qe - q0) * sum(parts[j][1] - parts[j][0] for j in ks)
+                     for k, ks in enumerate(sets) if plan2[t, k])
         n_tiles += 1
         if elapsed >= budget_s:
             break
     tflops = flops / elapsed / 1e12
     step_ms = counts["computed_flops"] / (flops / elapsed) * 1e3
+    ratio = counts["skipped_blocks"] / max(1, counts["skipped_blocks"] + counts["computed_blocks"])
+    layout = f", groups of {group}" if group else ""
     return {"tflops": tflops, "step_ms_extrapolated": step_ms, "threads": threads,
-            "sample": f"{n_tiles} query tiles x {len(hs)} head(s) of one {int(100 * r / w.P)}%-reuse step "
-                      f"({flops / 1e9:.1f} GFLOP, {elapsed:.1f} s), float64 numpy oracle"}
+            "sample": f"{n_tiles} query tiles x {len(hs)} head(s) of one {int(round(100 * ratio))}%-reuse step"
+                      f"{layout} ({flops / 1e9:.1f} GFLOP, {elapsed:.1f} s), float64 numpy oracle"}
 
 
-def run_reference(args, w, r, rank):
+def run_reference(args, w, r, rank, group=0):
     if rank != 0:
         return
     from partitioned_attention_state_b200 import workloads as wl
@@ -223,10 +230,10 @@ def run_reference(args, w, r, rank):
     inputs = s.next_step() + s.next_step()
     budget = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_sample(w, r, budget_s=budget * 0.25, inputs=inputs)
+        oracle_sample(w, r, budget_s=budget * 0.25, inputs=inputs, group=group)
     vals, samples = [], []
     for _ in range(args.steps):
-        res = oracle_sample(w, r, budget_s=budget, inputs=inputs)
+        res = oracle_sample(w, r, budget_s=budget, inputs=inputs, group=group)
         vals.append(res["tflops"])
         samples.append(res)
     v = float(np.mean(vals))
@@ -235,8 +242,8 @@ def run_reference(args, w, r, rank):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean([s["step_ms_extrapolated"] for s in samples])),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "H": w.H, "S": w.S, "D": w.D, "P": w.P, "reuse_per_row": r,
-                   "reuse_ratio": r / w.P},
+        "config": {"workload": w.name, "H": w.H, "S": w.S, "D": w.D, "P": w.P, "group": group, "reuse_per_row": r,
+                   "reuse_ratio": r / (w.P if group == 0 else -(-w.P // group))},
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": last["threads"], "kind": "oracle",
                          "sample": last["sample"]},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -256,12 +263,14 @@ def main():
     if args.heads is not None:
         import dataclasses
         w = dataclasses.replace(w, H=args.heads, name=f"{w.name}_h{args.heads}")
-    r = args.reuse if args.reuse is not None else (w.P // 2 if w.mode == "proximity" else 0)
+    grp = args.group if w.mode == "proximity" else 0
+    n_sets = w.P if grp == 0 else -(-w.P // grp)        # reusable key sets per query tile
+    r = args.reuse if args.reuse is not None else (n_sets // 2 if w.mode == "proximity" else 0)
 
     if args.impl == "reference":
         if world > 1 and rank != 0:
             return
-        run_reference(args, w, r, rank)
+        run_reference(args, w, r, rank, grp)
         return
 
     import torch
@@ -277,7 +286,7 @@ def main():
 
     win = w.mode == "window"
     sess = Session(w.H, w.S, w.D, w.P, mode=dt.DT_MODE_WINDOW if win else dt.DT_MODE_PROXIMITY, reuse_per_row=r,
-                   window=w.window)
+                   window=w.window, group=grp)
     stream = wl.stream_for(w)
     q1, k1, v1 = stream.next_step()
     sess.set_inputs(q1, k1, v1)
@@ -327,15 +336,15 @@ def main():
     pk, pk_kind = peaks()
     peak_tf = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (kern_ms * 1e-3) / 1e12
-    traffic = recorded_traffic(w.name, r)
+    traffic = recorded_traffic(w.name, r) if grp == 0 else None
 
     # reuse sweep 0/25/50/75 %
     sweep = None
     if not args.no_sweep and not win:
         sweep = {}
-        for rr in sorted({0, w.P // 4, w.P // 2, 3 * w.P // 4}):
+        for rr in sorted({0, n_sets // 4, n_sets // 2, 3 * n_sets // 4}):
             ms, km, c = timed(max(5, args.steps // 2), 3, rr)
-            sweep[f"{int(round(100 * rr / w.P))}%"] = {
+            sweep[f"{int(round(100 * rr / n_sets))}%"] = {
                 "reuse_per_row": rr, "ms_per_step": ms, "kernel_ms": km,
                 "tflops": c["computed_flops"] / (km * 1e-3) / 1e12,
                 "frac_of_peak": c["computed_flops"] / (km * 1e-3) / 1e12 / peak_tf,
@@ -344,7 +353,7 @@ def main():
 
     # standalone state merge over the whole cache (HBM-bound)
     merge = None
-    if not win:
+    if not win and grp == 0:
         o_out = torch.empty((w.H, w.S, w.D), dtype=torch.float32, device="cuda")
         l_out = torch.empty((w.H, w.S), dtype=torch.float32, device="cuda")
         for _ in range(3):
@@ -363,6 +372,55 @@ def main():
         merge = {"kernel": "state_merge", "ms": mms, "bytes": nbytes, "GB/s": nbytes / (mms * 1e-3) / 1e9,
                  "frac_of_hbm": nbytes / (mms * 1e-3) / 1e9 / hbm}
         del o_out, l_out
+
+    # the same step on the grouped cache (groups of 4 partitions, half of the
+    # groups reused), and the in-place regrouping of that cache 4 -> 8
+    grouped = compose = None
+    if not win and grp == 0 and not args.no_grouped and w.P % 4 == 0 and w.P >= 8:
+        g4, m4 = 4, w.P // 4
+        gs = Session(w.H, w.S, w.D, w.P, reuse_per_row=m4 // 2, group=g4)
+        gs.set_inputs(q1, k1, v1)
+        gs.step(1)
+        gs.set_inputs(q2, k2, v2)
+        gs.check()
+        graph = gs.capture_step(2)
+        for _ in range(3):
+            graph.replay()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ng = max(5, args.steps // 2)
+        a.record(cur)
+        for _ in range(ng):
+            gc = graph.replay()
+        b.record(cur)
+        barrier()
+        gs.check()
+        gms = max_over_ranks([a.elapsed_time(b) / ng], "cuda")[0]
+        slot_bytes = w.H * w.S * (4 * w.D + 4)
+        grouped = {"group": g4, "reuse_groups": m4 // 2, "cache_slots": 1 + m4,
+                   "cache_bytes": (1 + m4) * slot_bytes, "per_partition_cache_bytes": w.P * slot_bytes,
+                   "reuse_ratio": gc["skipped_blocks"] / (gc["skipped_blocks"] + gc["computed_blocks"]),
+                   "ms_per_step": gms, "tflops": gc["computed_flops"] / (gms * 1e-3) / 1e12,
+                   "frac_of_peak": gc["computed_flops"] / (gms * 1e-3) / 1e12 / peak_tf,
+                   "per_partition_ms_per_step": ms_step, "launch": "CUDA-graph replay"}
+        del graph
+        # regroup 4 -> 8 in place, repeatedly on the same buffers (HBM-bound)
+        pc = dt.params(w.H, w.S, w.D, w.P, dt.DT_MODE_PROXIMITY, 0, 0, 1, g4)
+        for _ in range(3):
+            dt.dt_group_compose(pc, 2, None, gs.cache_O, gs.cache_L, gs.status)
+        barrier()
+        a.record(cur)
+        nc = 5
+        for _ in range(nc):
+            dt.dt_group_compose(pc, 2, None, gs.cache_O, gs.cache_L, gs.status)
+        b.record(cur)
+        barrier()
+        cms = max_over_ranks([a.elapsed_time(b) / nc], "cuda")[0]
+        cbytes = (m4 + -(-m4 // 2)) * slot_bytes
+        hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        compose = {"kernel": "group_compose", "from_group": g4, "to_group": 2 * g4, "ms": cms, "bytes": cbytes,
+                   "GB/s": cbytes / (cms * 1e-3) / 1e9, "frac_of_hbm": cbytes / (cms * 1e-3) / 1e9 / hbm}
+        del gs
 
     # end to end through the public API with host buffers
     e2e = None
@@ -395,7 +453,7 @@ def main():
 
     cpu = None
     if rank == 0 and not args.no_cpu:
-        res = oracle_sample(w, r, budget_s=12.0, inputs=(q1, k1, v1, q2, k2, v2))
+        res = oracle_sample(w, r, budget_s=12.0, inputs=(q1, k1, v1, q2, k2, v2), group=grp)
         cpu = {"value": res["tflops"], "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
                "sample": res["sample"], "ms_per_step_extrapolated": res["step_ms_extrapolated"]}
 
@@ -405,7 +463,9 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "H": w.H, "S": w.S, "D": w.D, "P": w.P, "window": w.window,
-                       "reuse_per_row": r, "reuse_ratio": r / w.P, "step": "reuse step after an anchor step",
+                       "group": grp, "reuse_per_row": r,
+                       "reuse_ratio": counts["skipped_blocks"] / max(1, counts["skipped_blocks"] + counts["computed_blocks"]),
+                       "step": "reuse step after an anchor step",
                        "launch": "eager host path" if args.eager else "CUDA-graph replay of the fused launch",
                        "computed_blocks": counts["computed_blocks"], "skipped_blocks": counts["skipped_blocks"],
                        "computed_flops": flops, "parallelism": f"replicas x{world}",
@@ -420,6 +480,8 @@ def main():
             "cpu_baseline": cpu,
             "reuse_sweep": sweep,
             "state_merge": merge,
+            "grouped": grouped,
+            "group_compose": compose,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

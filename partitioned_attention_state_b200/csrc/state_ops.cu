@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(kBlock) window_residual_kernel(int op, int64_t
 // writes slot 1 + i, which only an already finished group read.  Inside a
 // group every lane reads all inputs (the LSEs are shared by the whole row)
 // before any lane writes, so the write of slot 1 + i cannot race a read of it.
+// F (>= factor) bounds the inputs a lane loads at once.
+template <int F>
 __global__ void __launch_bounds__(kBlock) group_compose_kernel(int m, int factor, int64_t rows, int D,
                                                                float* __restrict__ cO, float* __restrict__ cL) {
   const int lane = threadIdx.x & 31;
@@ -113,29 +115,51 @@ __global__ void __launch_bounds__(kBlock) group_compose_kernel(int m, int factor
   for (int64_t row = blockIdx.x * (int64_t)(kBlock / 32) + (threadIdx.x >> 5); row < rows; row += warps) {
     for (int i = 0; i < m2; ++i) {
       const int j0 = 1 + factor * i, n = min(factor, m - factor * i);
-      float M = kNegInf;
-      for (int k = 0; k < n; ++k) M = fmaxf(M, cL[(int64_t)(j0 + k) * rows + row]);
-      float Lr = kNegInf, tot = 0.f;
+      // all reads of this group first, issued together: the LSEs and this
+      // lane's OUT columns (a slot with LSE -inf gets weight 0 and its OUT,
+      // possibly never written, is replaced by zeros after the load)
+      float lv[F];
+      float4 v[F];
+      const bool one = d4n <= 32;               // D <= 128: one float4 per lane
+#pragma unroll
+      for (int k = 0; k < F; ++k) {
+        lv[k] = k < n ? cL[(int64_t)(j0 + k) * rows + row] : kNegInf;
+        v[k] = (one && k < n && lane < d4n)
+                   ? reinterpret_cast<const float4*>(cO + ((int64_t)(j0 + k) * rows + row) * D)[lane]
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float M = lv[0];
+#pragma unroll
+      for (int k = 1; k < F; ++k) M = fmaxf(M, lv[k]);
+      float w[F];
+      float Lr = kNegInf;
       if (M > kNegInf) {
-        for (int k = 0; k < n; ++k) tot += expf(cL[(int64_t)(j0 + k) * rows + row] - M);
+        float tot = 0.f;
+#pragma unroll
+        for (int k = 0; k < F; ++k) tot += k < n ? expf(lv[k] - M) : 0.f;
         Lr = M + logf(tot);
       }
-      float w[8];                               // factor <= 8 (checked on the host)
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        w[k] = (k < n && M > kNegInf) ? expf(cL[(int64_t)(j0 + k) * rows + row] - Lr) : 0.f;
-      // each lane composes its own columns: it reads them all before writing
+      for (int k = 0; k < F; ++k) w[k] = (k < n && lv[k] > kNegInf) ? expf(lv[k] - Lr) : 0.f;
       for (int c4 = lane; c4 < d4n; c4 += 32) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int k = 0; k < n; ++k) {
-          if (w[k] == 0.f) continue;
-          const float4 v = reinterpret_cast<const float4*>(cO + ((int64_t)(j0 + k) * rows + row) * D)[c4];
-          acc.x = fmaf(w[k], v.x, acc.x);
-          acc.y = fmaf(w[k], v.y, acc.y);
-          acc.z = fmaf(w[k], v.z, acc.z);
-          acc.w = fmaf(w[k], v.w, acc.w);
+        if (!one) {
+#pragma unroll
+          for (int k = 0; k < F; ++k)
+            v[k] = k < n ? reinterpret_cast<const float4*>(cO + ((int64_t)(j0 + k) * rows + row) * D)[c4]
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        reinterpret_cast<float4*>(cO + ((int64_t)(1 + i) * rows + row) * D)[c4] = acc;
+#pragma unroll
+        for (int k = 0; k < F; ++k)
+          if (w[k] == 0.f) v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < F; ++k) {
+          acc.x = fmaf(w[k], v[k].x, acc.x);
+          acc.y = fmaf(w[k], v[k].y, acc.y);
+          acc.z = fmaf(w[k], v[k].z, acc.z);
+          acc.w = fmaf(w[k], v[k].w, acc.w);
+        }
+        __stcs(reinterpret_cast<float4*>(cO + ((int64_t)(1 + i) * rows + row) * D) + c4, acc);
       }
       __syncwarp();                             // every lane has read this group's LSEs
       if (lane == 0) cL[(int64_t)(1 + i) * rows + row] = Lr;
@@ -170,7 +194,13 @@ int launch_cache_update(const Geom& G, const uint8_t* plan, const float* fO, con
 
 int launch_group_compose(int m, int factor, int H, int S, int D, float* cO, float* cL, int sms, cudaStream_t st) {
   const int64_t rows = (int64_t)H * S;
-  group_compose_kernel<<<grid_for(rows * 32, sms), kBlock, 0, st>>>(m, factor, rows, D, cO, cL);
+  const int grid = grid_for(rows * 32, sms);
+  switch (factor) {   // the factor bounds how many inputs a lane loads at once
+    case 2: group_compose_kernel<2><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL); break;
+    case 3: group_compose_kernel<3><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL); break;
+    case 4: group_compose_kernel<4><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL); break;
+    default: group_compose_kernel<8><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL); break;   // 5..8
+  }
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
 }
 
