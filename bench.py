@@ -98,10 +98,11 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, r):
+def recorded_traffic(workload, r, group=0):
     """DRAM bytes per launch of the fused kernel from a committed ncu summary,
     valid only while the kernel sources are unchanged since the capture."""
-    path = os.path.join(ROOT, "profiles", f"attn_fused_sm100_{workload}.md")
+    suffix = f"_g{group}" if group else ""
+    path = os.path.join(ROOT, "profiles", f"attn_fused_sm100_{workload}{suffix}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -336,7 +337,7 @@ def main():
     pk, pk_kind = peaks()
     peak_tf = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (kern_ms * 1e-3) / 1e12
-    traffic = recorded_traffic(w.name, r) if grp == 0 else None
+    traffic = recorded_traffic(w.name, r, grp)
 
     # reuse sweep 0/25/50/75 %
     sweep = None
