@@ -57,7 +57,8 @@ def parse_args():
     ap.add_argument("--heads", type=int, default=None, help="override H (smaller profiling captures)")
     ap.add_argument("--group", type=int, default=0,
                     help="state grouping: groups of G adjacent partitions, --reuse then counts groups")
-    ap.add_argument("--no-grouped", action="store_true", help="skip the grouped-cache and compose measurements")
+    ap.add_argument("--no-grouped", action="store_true",
+                    help="skip the grouped-cache, compose and bf16-cache measurements")
     return ap.parse_args()
 
 
@@ -376,27 +377,44 @@ def main():
 
     # the same step on the grouped cache (groups of 4 partitions, half of the
     # groups reused), and the in-place regrouping of that cache 4 -> 8
-    grouped = compose = None
-    if not win and grp == 0 and not args.no_grouped and w.P % 4 == 0 and w.P >= 8:
-        g4, m4 = 4, w.P // 4
-        gs = Session(w.H, w.S, w.D, w.P, reuse_per_row=m4 // 2, group=g4)
-        gs.set_inputs(q1, k1, v1)
-        gs.step(1)
-        gs.set_inputs(q2, k2, v2)
-        gs.check()
-        graph = gs.capture_step(2)
+    def time_session(vs):
+        """Anchor, then the graph-replayed reuse step of another session over
+        the same inputs: (ms per step, counts)."""
+        vs.set_inputs(q1, k1, v1)
+        vs.step(1)
+        vs.set_inputs(q2, k2, v2)
+        vs.check()
+        graph = vs.capture_step(2)
         for _ in range(3):
             graph.replay()
         barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ng = max(5, args.steps // 2)
+        n = max(5, args.steps // 2)
         a.record(cur)
-        for _ in range(ng):
-            gc = graph.replay()
+        for _ in range(n):
+            vc = graph.replay()
         b.record(cur)
         barrier()
-        gs.check()
-        gms = max_over_ranks([a.elapsed_time(b) / ng], "cuda")[0]
+        vs.check()
+        del graph
+        return max_over_ranks([a.elapsed_time(b) / n], "cuda")[0], vc
+
+    grouped = compose = bf16c = None
+    if not win and grp == 0 and not args.no_grouped:
+        # the same step with the cached OUT stored in bf16
+        bs = Session(w.H, w.S, w.D, w.P, reuse_per_row=r, state_dtype=dt.DT_STATE_BF16)
+        bms, bc = time_session(bs)
+        bf16c = {"state_dtype": "bf16 OUT, fp32 LSE", "cache_bytes": w.P * w.H * w.S * (2 * w.D + 4),
+                 "fp32_cache_bytes": w.P * w.H * w.S * (4 * w.D + 4), "ms_per_step": bms,
+                 "tflops": bc["computed_flops"] / (bms * 1e-3) / 1e12,
+                 "frac_of_peak": bc["computed_flops"] / (bms * 1e-3) / 1e12 / peak_tf,
+                 "fp32_ms_per_step": ms_step, "launch": "CUDA-graph replay"}
+        del bs
+    if not win and grp == 0 and not args.no_grouped and w.P % 4 == 0 and w.P >= 8:
+        g4, m4 = 4, w.P // 4
+        gs = Session(w.H, w.S, w.D, w.P, reuse_per_row=m4 // 2, group=g4)
+        gms, gc = time_session(gs)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         slot_bytes = w.H * w.S * (4 * w.D + 4)
         grouped = {"group": g4, "reuse_groups": m4 // 2, "cache_slots": 1 + m4,
                    "cache_bytes": (1 + m4) * slot_bytes, "per_partition_cache_bytes": w.P * slot_bytes,
@@ -404,7 +422,6 @@ def main():
                    "ms_per_step": gms, "tflops": gc["computed_flops"] / (gms * 1e-3) / 1e12,
                    "frac_of_peak": gc["computed_flops"] / (gms * 1e-3) / 1e12 / peak_tf,
                    "per_partition_ms_per_step": ms_step, "launch": "CUDA-graph replay"}
-        del graph
         # regroup 4 -> 8 in place, repeatedly on the same buffers (HBM-bound)
         pc = dt.params(w.H, w.S, w.D, w.P, dt.DT_MODE_PROXIMITY, 0, 0, 1, g4)
         for _ in range(3):
@@ -483,6 +500,7 @@ def main():
             "state_merge": merge,
             "grouped": grouped,
             "group_compose": compose,
+            "bf16_state_cache": bf16c,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -82,7 +82,13 @@ typedef struct {
   int32_t step;                 /* denoising step t, 1-based; step 1 is an anchor */
   int32_t group;                /* g: 0 = one key set per partition; g >= 1 = state grouping (below).
                                    Partition modes only (0 in window mode) */
+  int32_t state_dtype;          /* element type of the cached OUT: DT_STATE_F32 or DT_STATE_BF16
+                                   (partition modes; cached LSE is always fp32) */
 } dt_plan_params;
+
+#define DT_STATE_F32  0         /* cache_O is float [nseg][H][S][D] */
+#define DT_STATE_BF16 1         /* cache_O is bf16 [nseg][H][S][D] (RNE from the fp32 state),
+                                   half the bytes; accepted by dt_attn_partial_fused(_heads) only */
 
 /* State grouping ("DiTango", grouping of spatially adjacent attention states;
  * the local state is handled separately): with group size g the P partitions
@@ -185,7 +191,8 @@ DT_API int dt_state_merge(int32_t N, int32_t H, int32_t S, int32_t D,
  * computed states are stored in the attention state cache): for every
  * (query tile, partition k) with plan COMPUTE, copy the tile's rows of
  * fresh_O/fresh_L (layout of cache_O/cache_L) into cache_O/cache_L; REUSE
- * slots stay byte-identical.  Partition modes only.  HBM-bound kernel. */
+ * slots stay byte-identical.  Partition modes and fp32 states only
+ * (DT_ERR_UNSUPPORTED for DT_STATE_BF16).  HBM-bound kernel. */
 DT_API int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_plan,
                           const float* fresh_O, const float* fresh_L,
                           float* cache_O, float* cache_L,
@@ -201,8 +208,8 @@ DT_API int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_plan,
  * with p->group = g*factor.  stamps (host, optional) is [nqt][1+m] on entry
  * and is rewritten as [nqt][1+m'] in its first entries: a composed slot gets
  * the oldest stamp of the slots it merges (-1 if any is -1).  One launch of an
- * HBM-bound kernel.  Errors: DT_ERR_INVALID (bad params, factor < 2, null
- * cache), DT_ERR_UNSUPPORTED (misaligned cache pointers). */
+ * HBM-bound kernel.  Errors: DT_ERR_INVALID (bad params, factor < 2 or > 8,
+ * null cache), DT_ERR_UNSUPPORTED (misaligned cache pointers, bf16 states). */
 DT_API int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t* stamps,
                      float* cache_O, float* cache_L, int32_t* d_status, void* stream);
 

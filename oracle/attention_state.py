@@ -35,6 +35,8 @@ notes of the repository):
     cached per (query tile, key set) and the plan decides per key set; the
     proximity plan reuses the r groups farthest from q's group (lower index
     first among equal distances) and always computes {q};
+  * a bf16 state cache stores OUT rounded to nearest-even bf16 and LSE in
+    float64 (fp32 on the GPU);
   * Dynamic Group State Compose by a factor k: the new group i is old groups
     k i .. k i + k - 1, its cached state their composition, its stamp the
     oldest of theirs (never written if any was never written).
@@ -347,17 +349,22 @@ def build_plan(mode: int, H: int, S: int, D: int, P: int, step: int,
 # ----------------------------------------------------------------------------
 
 class StateCache:
-    """Per-(KV partition, head) cached states of query rows.
+    """Per-(key set, head) cached states of query rows.
 
-    ``out[k][h]`` is a dict row -> (OUT [D], LSE) for the rows tracked.  Rows
-    are independent, so a sampled subset of rows can be followed through a
-    whole schedule exactly.
+    ``slots[(k, h, row)]`` = (OUT [D], LSE) for the rows tracked.  Rows are
+    independent, so a sampled subset of rows can be followed through a whole
+    schedule exactly.  With ``bf16`` the stored OUT is rounded to the nearest
+    bf16 value (ties to even), the storage form the pages' memory argument
+    assumes (a state is half the size of its partition's KV); LSE is kept
+    exactly.
     """
 
-    def __init__(self):
+    def __init__(self, bf16: bool = False):
         self.slots: Dict[Tuple[int, int, int], Tuple[np.ndarray, float]] = {}
+        self.bf16 = bf16
 
     def put(self, k, h, rows, out, lse):
+        out = round_bf16(out) if self.bf16 else out
         for i, r in enumerate(rows):
             self.slots[(k, h, int(r))] = (out[i].copy(), float(lse[i]))
 

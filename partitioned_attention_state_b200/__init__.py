@@ -24,10 +24,11 @@ __all__ = [
     "DT_OK", "DT_ERR_INVALID", "DT_ERR_UNSUPPORTED", "DT_ERR_CACHE_EMPTY", "DT_ERR_CUDA",
     "DT_ERR_TIMEOUT", "DT_MODE_ALL_COMPUTE", "DT_MODE_PROXIMITY", "DT_MODE_ALL_REUSE",
     "DT_MODE_EXPLICIT", "DT_MODE_WINDOW", "DT_PLAN_REUSE", "DT_PLAN_COMPUTE", "DT_WR_MAKE",
-    "DT_WR_APPLY", "DT_TILE",
+    "DT_WR_APPLY", "DT_TILE", "DT_STATE_F32", "DT_STATE_BF16",
 ]
 
 DT_OK, DT_ERR_INVALID, DT_ERR_UNSUPPORTED, DT_ERR_CACHE_EMPTY, DT_ERR_CUDA, DT_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+DT_STATE_F32, DT_STATE_BF16 = 0, 1
 DT_MODE_ALL_COMPUTE, DT_MODE_PROXIMITY, DT_MODE_ALL_REUSE, DT_MODE_EXPLICIT, DT_MODE_WINDOW = 0, 1, 2, 3, 4
 DT_PLAN_REUSE, DT_PLAN_COMPUTE = 0, 1
 DT_WR_MAKE, DT_WR_APPLY = 0, 1
@@ -43,7 +44,7 @@ class DtError(RuntimeError):
 class PlanParams(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int32), ("S", ctypes.c_int32), ("D", ctypes.c_int32), ("P", ctypes.c_int32),
                 ("mode", ctypes.c_int32), ("reuse_per_row", ctypes.c_int32), ("window", ctypes.c_int32),
-                ("step", ctypes.c_int32), ("group", ctypes.c_int32)]
+                ("step", ctypes.c_int32), ("group", ctypes.c_int32), ("state_dtype", ctypes.c_int32)]
 
 
 class Plan(ctypes.Structure):
@@ -114,8 +115,9 @@ def dt_status_string(status: int) -> str:
     return load().dt_status_string(status).decode()
 
 
-def params(H, S, D, P=1, mode=DT_MODE_ALL_COMPUTE, reuse_per_row=0, window=0, step=1, group=0) -> PlanParams:
-    return PlanParams(H, S, D, P, mode, reuse_per_row, window, step, group)
+def params(H, S, D, P=1, mode=DT_MODE_ALL_COMPUTE, reuse_per_row=0, window=0, step=1, group=0,
+           state_dtype=0) -> PlanParams:
+    return PlanParams(H, S, D, P, mode, reuse_per_row, window, step, group, state_dtype)
 
 
 def dt_plan_geometry(p: PlanParams):

@@ -84,6 +84,8 @@ extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head
   if (!shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (win ? p->window < 1 : p->P < 1) return DT_ERR_INVALID;
   if (p->group < 0 || (win && p->group != 0)) return DT_ERR_INVALID;
+  if (p->state_dtype != DT_STATE_F32 && p->state_dtype != DT_STATE_BF16) return DT_ERR_INVALID;
+  if (win && p->state_dtype != DT_STATE_F32) return DT_ERR_INVALID;
   if (head_begin < 0 || head_count < 0 || head_begin > p->H - head_count) return DT_ERR_INVALID;
   if (p->D != 64 && p->D != 72 && p->D != 128) return DT_ERR_UNSUPPORTED;
   const int nseg = win ? 2 : (p->group > 0 ? 1 + dt::ceil_div(p->P, p->group) : p->P);
@@ -121,6 +123,7 @@ extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head
   kp.status = d_status;
   kp.H = p->H; kp.S = p->S; kp.D = p->D; kp.P = win ? 1 : p->P; kp.window = win ? p->window : 0;
   kp.geom = G;
+  kp.state_bf16 = p->state_dtype == DT_STATE_BF16;
   // items are numbered over all heads, so a head range computes exactly what
   // the whole launch computes for those heads
   kp.item0 = head_begin * G.nqt;
@@ -162,6 +165,7 @@ extern "C" int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_p
   if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW)
     return DT_ERR_INVALID;
   if (p->P < 1 || p->group < 0 || p->D < 4 || p->D % 4 != 0 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
+  if (p->state_dtype != DT_STATE_F32) return DT_ERR_UNSUPPORTED;
   if (p->H == 0 || p->S == 0) return DT_OK;
   if (!d_plan || !fresh_O || !fresh_L || !cache_O || !cache_L) return DT_ERR_INVALID;
   if (!aligned16(fresh_O) || !aligned16(cache_O) || !aligned16(fresh_L) || !aligned16(cache_L))
@@ -179,6 +183,7 @@ extern "C" int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t
   if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW)
     return DT_ERR_INVALID;
   if (p->P < 1 || p->group < 1 || factor < 2 || factor > 8) return DT_ERR_INVALID;
+  if (p->state_dtype != DT_STATE_F32) return DT_ERR_UNSUPPORTED;
   if (p->D < 4 || p->D % 4 != 0 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if ((int64_t)p->group * factor > (int64_t)1 << 30) return DT_ERR_INVALID;
   const dt::Geom G = dt::make_geom(p->H, p->S, p->D, p->P, 0, p->group);

@@ -23,6 +23,7 @@ struct AttnParams {
   int H, S, D, P, window;           // P: partitions (ignored in window mode)
   Geom geom;                        // make_geom(H, S, D, P, window), read from the parameter bank
   int item0, item_end;              // items [item0, item_end) of the H * nqt (head-major) items
+  int state_bf16;                   // cached OUT is bf16 (cache_O then points to bf16 data)
   float scale_log2;                 // log2(e) / sqrt(D)
   uint64_t wait_limit_ns;
 };

@@ -247,10 +247,16 @@ __device__ __forceinline__ bool issue_pv(uint64_t* bars, uint32_t tmem, uint32_t
   return true;
 }
 
+// MODE: key-set mode (kModePartition, kModeWindow, kModeGrouped) in bits 0-1,
+// kStateBf16 when the cached OUT is bf16 (partition modes).
+constexpr int kStateBf16 = 4;
+
 template <int DP, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const __grid_constant__ AttnParams p) {
   using C = Cfg<DP>;
-  constexpr bool WIN = MODE == kModeWindow;
+  constexpr int KM = MODE & 3;
+  constexpr bool WIN = KM == kModeWindow;
+  constexpr bool CBF = (MODE & kStateBf16) != 0;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {                       // layout needs 1024-byte alignment
     if (threadIdx.x == 0) atomicCAS(p.status, 0, DT_ERR_UNSUPPORTED);
@@ -316,9 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
-        if (!item_has_compute<MODE>(G, qt, cm)) continue;
+        if (!item_has_compute<KM>(G, qt, cm)) continue;
         if (is_k) {
-          const QTile t = query_tile<MODE>(G, qt);
+          const QTile t = query_tile<KM>(G, qt);
           if (nq > 0 && !mbar_wait(&bars[C::bQEmpty], (nq - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
             goto tma_done;
           mbar_arrive_expect_tx(&bars[C::bQFull], C::kTileBytes);
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         for (int j = 0; j < G.P; ++j) {
           const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
-          const KeySet ks = key_set<MODE>(G, qt, seg);
+          const KeySet ks = key_set<KM>(G, qt, seg);
           const int nt = ks.ntiles();
           const int toff = nt > 0 ? tile_rotation(nt, idx, seg) : 0;
           for (int i = 0; i < nt; ++i, ++g) {
@@ -374,14 +380,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
-        if (!item_has_compute<MODE>(G, qt, cm)) continue;
+        if (!item_has_compute<KM>(G, qt, cm)) continue;
         if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
         ++nq;
         tc_fence_after();
         for (int j = 0; j < G.P && ok; ++j) {
           const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
-          const int nt = key_set<MODE>(G, qt, seg).ntiles();
+          const int nt = key_set<KM>(G, qt, seg).ntiles();
           if (nt == 0) continue;
           for (int i = 0; i < nt; ++i, ++g) {
             const int st = g % C::kStages;
@@ -446,11 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const int qt = idx - (idx / G.nqt) * G.nqt;
         const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
         const int rot = seg_rotation<WIN>(G, idx);
-        if (!item_has_compute<MODE>(G, qt, cm)) continue;
+        if (!item_has_compute<KM>(G, qt, cm)) continue;
         for (int j = 0; j < G.P && ok; ++j) {
           const int seg = visit_seg<WIN>(G, rot, j);
           if (!is_compute(cm, seg)) continue;
-          const int nt = key_set<MODE>(G, qt, seg).ntiles();
+          const int nt = key_set<KM>(G, qt, seg).ntiles();
           if (nt == 0) continue;
           for (int i = 0; i < nt && ok; ++i, ++g)
             ok = issue_pv<DP>(bars, tmem, aV, g, cseg, i == 0, i == nt - 1, WIN && seg == 0, abort_flag, p.status,
@@ -481,14 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const int qt = idx - (idx / G.nqt) * G.nqt;
       const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
       const int rot = seg_rotation<WIN>(G, idx);
-      if (!item_has_compute<MODE>(G, qt, cm)) continue;
-      const QTile t = query_tile<MODE>(G, qt);
+      if (!item_has_compute<KM>(G, qt, cm)) continue;
+      const QTile t = query_tile<KM>(G, qt);
       const int qa = t.q0 + ra, qb = t.q0 + rb;
       const int q1 = t.q0 + t.rows - 1;
       for (int j = 0; j < G.P; ++j) {
         const int seg = visit_seg<WIN>(G, rot, j);
         if (!is_compute(cm, seg)) continue;
-        const KeySet ks = key_set<MODE>(G, qt, seg);
+        const KeySet ks = key_set<KM>(G, qt, seg);
         const int nt = ks.ntiles();
         if (nt == 0) continue;
         const int toff = tile_rotation(nt, idx, seg);
@@ -668,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       const int h = idx / G.nqt, qt = idx - (idx / G.nqt) * G.nqt;
       const uint64_t cm = plan_mask<WIN>(p.plan + (size_t)qt * G.P, G.P);
       const int rot = seg_rotation<WIN>(G, idx);
-      const QTile t = query_tile<MODE>(G, qt);
+      const QTile t = query_tile<KM>(G, qt);
       const int qrow = t.q0 + r;
       const bool valid = r < t.rows;
       float m_tot = kNegInf, l_tot = 0.f;
@@ -688,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         for (; jr < G.P; ++jr) {
           const int seg = visit_seg<WIN>(G, rot, jr);
           if (is_compute(cm, seg)) continue;
-          n_skip += counted_blocks<MODE>(G, qt, seg);   // same in every lane; thread 0 reports
+          n_skip += counted_blocks<KM>(G, qt, seg);   // same in every lane; thread 0 reports
           ++n_read;
           if (WIN) { use_r = true; ++merged; continue; }   // complement reused: add R at the end
           const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
@@ -704,13 +710,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           }
           const float l_new = a * l_tot + b;
           const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
+          const uint4* srch = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.cache_O) + slot * D);
           const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 1
           for (int c1 = 0; c1 < D; c1 += 32) {             // 32 cached columns in flight together
             float4 cv[8];
+            if (CBF) {                                     // bf16 OUT: 8 columns per 16-byte load
+              uint4 hv[4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              cv[c] = (c1 + 4 * c < D && valid && nonempty) ? __ldcs(src + c1 / 4 + c) : z4;
+              for (int c = 0; c < 4; ++c)
+                hv[c] = (c1 + 8 * c < D && valid && nonempty) ? __ldcs(srch + c1 / 8 + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                cv[2 * c] = make_float4(bf16lo(hv[c].x), bf16hi(hv[c].x), bf16lo(hv[c].y), bf16hi(hv[c].y));
+                cv[2 * c + 1] = make_float4(bf16lo(hv[c].z), bf16hi(hv[c].z), bf16lo(hv[c].w), bf16hi(hv[c].w));
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                cv[c] = (c1 + 4 * c < D && valid && nonempty) ? __ldcs(src + c1 / 4 + c) : z4;
+            }
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               if (c1 + 4 * c < D) {
@@ -733,14 +752,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       for (int j = 0; j < G.P; ++j) {
         const int seg = visit_seg<WIN>(G, rot, j);
         if (!is_compute(cm, seg)) continue;
-        const int nt = key_set<MODE>(G, qt, seg).ntiles();
+        const int nt = key_set<KM>(G, qt, seg).ntiles();
         const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
-        n_comp += counted_blocks<MODE>(G, qt, seg);
+        n_comp += counted_blocks<KM>(G, qt, seg);
         ++n_fresh;
         if (nt == 0) {             // empty key set: the identity state
           if (!WIN && valid) {
-            float4* dst = reinterpret_cast<float4*>(p.cache_O + slot * D);
-            for (int d = 0; d < D / 4; ++d) __stcs(dst + d, make_float4(0.f, 0.f, 0.f, 0.f));
+            if (CBF) {
+              uint2* dst = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.cache_O) + slot * D);
+              for (int d = 0; d < D / 4; ++d) __stcs(dst + d, make_uint2(0, 0));
+            } else {
+              float4* dst = reinterpret_cast<float4*>(p.cache_O + slot * D);
+              for (int d = 0; d < D / 4; ++d) __stcs(dst + d, make_float4(0.f, 0.f, 0.f, 0.f));
+            }
             __stcs(p.cache_L + slot, kNegInf);
           }
           continue;
@@ -785,7 +809,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             orow[(c + k) * 128] = nw[k];
           }
           if (valid) {
-            if (!WIN) {
+            if (!WIN && CBF) {
+              uint2 pk;
+              pk.x = pack_bf16x2(x[0] * inv_l, x[1] * inv_l);
+              pk.y = pack_bf16x2(x[2] * inv_l, x[3] * inv_l);
+              __stcs(reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.cache_O) + slot * D + c), pk);
+            } else if (!WIN) {
               __stcs(reinterpret_cast<float4*>(p.cache_O + slot * D + c),
                      make_float4(x[0] * inv_l, x[1] * inv_l, x[2] * inv_l, x[3] * inv_l));
             } else if (make_r) {
@@ -876,8 +905,11 @@ int attn_fused_smem_bytes(int dp) {
 template <int DP>
 int launch_mode(const AttnParams& kp, int grid, cudaStream_t stream) {
   if (kp.window > 0) return launch_dp<DP, kModeWindow>(kp, grid, stream);
-  if (kp.geom.grp > 0) return launch_dp<DP, kModeGrouped>(kp, grid, stream);
-  return launch_dp<DP, kModePartition>(kp, grid, stream);
+  if (kp.geom.grp > 0)
+    return kp.state_bf16 ? launch_dp<DP, kModeGrouped | kStateBf16>(kp, grid, stream)
+                         : launch_dp<DP, kModeGrouped>(kp, grid, stream);
+  return kp.state_bf16 ? launch_dp<DP, kModePartition | kStateBf16>(kp, grid, stream)
+                       : launch_dp<DP, kModePartition>(kp, grid, stream);
 }
 
 int launch_attn_fused(const AttnParams& kp, int dp, int grid, cudaStream_t stream) {

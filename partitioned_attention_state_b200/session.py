@@ -28,13 +28,16 @@ def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
 
 class Session:
     def __init__(self, H: int, S: int, D: int, P: int = 1, mode: int = DT_MODE_PROXIMITY, reuse_per_row: int = 0,
-                 window: int = 0, device: str = "cuda", cache: bool = True, group: int = 0):
+                 window: int = 0, device: str = "cuda", cache: bool = True, group: int = 0,
+                 state_dtype: int = 0):
         """group: 0 = one key set (and cache slot) per partition; g >= 1 =
         state grouping (the local partition, then groups of g adjacent
-        partitions); reuse_per_row then counts groups."""
+        partitions); reuse_per_row then counts groups.  state_dtype:
+        DT_STATE_F32 or DT_STATE_BF16 (cached OUT in bf16, half the bytes)."""
         self.H, self.S, self.D, self.P = H, S, D, P
         self.mode, self.r, self.window = mode, reuse_per_row, window
         self.group = group
+        self.state_dtype = state_dtype
         self.device = torch.device(device)
         win = mode == DT_MODE_WINDOW
         p = params(H, S, D, P if not win else 1, mode, reuse_per_row, window, 1, group)
@@ -50,7 +53,8 @@ class Session:
             self.R = torch.zeros((H, S, D), dtype=torch.float32, device=dev)
         else:
             ns = self.nseg
-            self.cache_O = torch.zeros((ns, H, S, D), dtype=torch.float32, device=dev) if cache else None
+            odt = torch.bfloat16 if state_dtype == 1 else torch.float32
+            self.cache_O = torch.zeros((ns, H, S, D), dtype=odt, device=dev) if cache else None
             self.cache_L = torch.full((ns, H, S), float("-inf"), dtype=torch.float32, device=dev) if cache else None
             self.R = None
         self._plan_buffers()
@@ -74,8 +78,8 @@ class Session:
         groups `factor` times coarser (in place on the device, stamps on the
         host); later steps plan on the coarser groups.  ``shrink`` moves the
         cache into buffers of the new size (a copy) to give memory back."""
-        if self.group < 1 or self.cache_O is None:
-            raise ValueError("compose_groups needs a grouped session with a cache")
+        if self.group < 1 or self.cache_O is None or self.state_dtype != 0:
+            raise ValueError("compose_groups needs a grouped session with an fp32 cache")
         p = params(self.H, self.S, self.D, self.P, self.mode, self.r, 0, 1, self.group)
         for ev in self._uploaded:
             if ev is not None:
@@ -102,7 +106,7 @@ class Session:
         mode = self.mode if mode is None else mode
         win = mode == DT_MODE_WINDOW
         p = params(self.H, self.S, self.D, 1 if win else self.P, mode, self.r, self.window, step,
-                   0 if win else self.group)
+                   0 if win else self.group, 0 if win else self.state_dtype)
         plan, counts = dt_plan_build(p, self.stamps, explicit)
         return p, plan, counts
 

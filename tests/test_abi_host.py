@@ -246,3 +246,22 @@ def test_group_compose_validated():
     p.D = 64
     assert lib.dt_group_compose(ctypes.byref(p), 2, None, 16 * 1024 + 4, 16 * 1024, None, None) == \
         dt.DT_ERR_UNSUPPORTED
+
+
+
+def test_state_dtype_validated():
+    import ctypes
+    lib = dt.load()
+    p = dt.params(1, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1, 0, 2)          # unknown state type
+    assert lib.dt_attn_partial_fused(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_INVALID
+    pw = dt.params(1, 1024, 64, 1, dt.DT_MODE_WINDOW, 0, 64, 1, 0, dt.DT_STATE_BF16)   # no cache in window mode
+    assert lib.dt_attn_partial_fused(ctypes.byref(pw), *([None] * 11), None) == dt.DT_ERR_INVALID
+    pb = dt.params(1, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1, 0, dt.DT_STATE_BF16)
+    assert lib.dt_attn_partial_fused(ctypes.byref(pb), *([None] * 11), None) == dt.DT_ERR_INVALID  # null buffers
+    assert lib.dt_state_cache_update(ctypes.byref(pb), *([None] * 7)) == dt.DT_ERR_UNSUPPORTED
+    pb.group = 2
+    assert lib.dt_group_compose(ctypes.byref(pb), 2, None, None, None, None, None) == dt.DT_ERR_UNSUPPORTED
+    # the plan does not depend on the state type
+    a, ca = dt.dt_plan_build(dt.params(1, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1), None)
+    b, cb = dt.dt_plan_build(dt.params(1, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1, 0, dt.DT_STATE_BF16), None)
+    assert np.array_equal(a, b) and ca == cb

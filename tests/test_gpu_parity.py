@@ -30,13 +30,13 @@ def _gpu():
 
 
 def run_partition_schedule(H, S, D, P, schedule, inputs, heads=None, rows=None, check_untouched=False,
-                           output_scaled=False, group=0, sess=None, cache=None):
+                           output_scaled=False, group=0, sess=None, cache=None, state_dtype=0):
     """schedule: list of (step, mode, r, explicit); inputs: callable -> (q,k,v) bits.
     group > 0: grouped key sets (one cache slot per group).  A session and
     oracle cache may be passed in to continue an earlier schedule."""
     if sess is None:
-        sess = Session(H, S, D, P, mode=dt.DT_MODE_PROXIMITY, group=group)
-        cache = orc.StateCache()
+        sess = Session(H, S, D, P, mode=dt.DT_MODE_PROXIMITY, group=group, state_dtype=state_dtype)
+        cache = orc.StateCache(bf16=state_dtype == dt.DT_STATE_BF16)
     group = sess.group
     hs = list(range(H)) if heads is None else list(heads)
     rs = np.arange(S) if rows is None else np.asarray(rows)
@@ -372,3 +372,31 @@ def test_group_compose_matches_oracle(P, g, f):
         np.testing.assert_allclose(got_l, want_l, rtol=0, atol=2e-5)
     run_partition_schedule(H, S, D, P, [(3, dt.DT_MODE_PROXIMITY, 1, None), (4, dt.DT_MODE_ALL_REUSE, 0, None)], s,
                            sess=sess, cache=new_cache)
+
+
+
+# ------------------------------------------------------------ bf16 state cache
+
+@pytest.mark.parametrize("H,S,D,P,g,rs", [
+    (16, 1024, 72, 8, 0, (4, 2, 6)),     # DiT-XL/2-like geometry
+    (2, 1024, 64, 4, 0, (2, 1)),
+    (2, 2600, 128, 7, 0, (3, 5)),        # D = 128, ragged partitions
+    (2, 2048, 128, 16, 4, (2, 1, 3)),    # with grouping
+    (1, 1800, 72, 12, 5, (1, 2)),
+])
+def test_bf16_state_cache_schedule_parity(H, S, D, P, g, rs):
+    """The bf16 state cache: fresh states are stored rounded to bf16 and
+    reused from there; outputs, cached states and untouched slots match the
+    oracle run with the same rounding of its cache."""
+    sched = [(1, dt.DT_MODE_PROXIMITY, rs[0], None)] + \
+            [(t + 2, dt.DT_MODE_PROXIMITY, r, None) for t, r in enumerate(rs)]
+    sess, _ = run_partition_schedule(H, S, D, P, sched, stream_of(H, S, D, 0.05, seed=S + 7), check_untouched=True,
+                                     group=g, state_dtype=dt.DT_STATE_BF16)
+    assert sess.cache_O.dtype == torch.bfloat16
+
+
+def test_bf16_state_cache_video_full_size_sampled_rows():
+    w = wl.WORKLOADS[3]
+    sched = [(1, dt.DT_MODE_PROXIMITY, 8, None), (2, dt.DT_MODE_PROXIMITY, 8, None)]
+    run_partition_schedule(w.H, w.S, w.D, w.P, sched, wl.stream_for(w).next_step, heads=[0, 39],
+                           rows=sample_rows(w.S, w.P, n_extra=16), state_dtype=dt.DT_STATE_BF16)

@@ -197,3 +197,41 @@ def test_compose_groups_stamp_is_oldest():
     st = np.array([[5, 3, 4, -1, 2, 7]], dtype=np.int32)    # 1 tile, local + 5 groups
     _, st2 = orc.compose_groups(orc.StateCache(), st, 5, 1, 2, [], np.zeros(0, int), 128, 4)
     assert st2.tolist() == [[5, 3, -1, 7]]
+
+
+# ------------------------------------------------------------ bf16 state cache
+
+def test_bf16_cache_stores_representable_values_and_exact_lse():
+    H, S, D, P = 1, 300, 8, 3
+    q, k, v = wl.InputStream(H, S, D, sigma=0.05, seed=50).next_step()
+    c32, c16 = orc.StateCache(), orc.StateCache(bf16=True)
+    plan, _, _ = orc.build_plan(orc.MODE_ALL_COMPUTE, H, S, D, P, step=1)
+    o32, l32, _ = orc.partition_step(q, k, v, plan, S, P, c32)
+    o16, l16, _ = orc.partition_step(q, k, v, plan, S, P, c16)
+    np.testing.assert_array_equal(o16, o32)            # the step's own output is not rounded
+    for key, (o, l) in c16.slots.items():
+        o_ref, l_ref = c32.slots[key]
+        assert l == l_ref
+        # every stored value is a bf16 value (8 significant bits) ...
+        m, e = np.frexp(o)
+        np.testing.assert_array_equal(np.ldexp(np.round(np.ldexp(m, 8)), e - 8), o)
+        # ... within half a bf16 spacing of the exact one
+        assert np.all(np.abs(o - o_ref) <= np.abs(o_ref) * 2.0 ** -8 + 1e-300)
+
+
+def test_bf16_cache_reuse_error_within_rounding_bound():
+    """With a bf16 cache and unchanged inputs, an all-REUSE step is a convex
+    combination of states whose OUT elements each carry a rounding error of
+    at most half a bf16 spacing, <= 2^-8 |x|, so it stays within 2^-8 max|OUT|
+    of full attention."""
+    H, S, D, P = 2, 640, 8, 5
+    q, k, v = wl.InputStream(H, S, D, sigma=0.0, seed=51).next_step()
+    cache = orc.StateCache(bf16=True)
+    plan, _, st = orc.build_plan(orc.MODE_ALL_COMPUTE, H, S, D, P, step=1)
+    full, lfull, _ = orc.partition_step(q, k, v, plan, S, P, cache)
+    plan2, _, _ = orc.build_plan(orc.MODE_ALL_REUSE, H, S, D, P, step=2, stamps=st)
+    o, l, _ = orc.partition_step(q, k, v, plan2, S, P, cache)
+    np.testing.assert_allclose(l, lfull, rtol=1e-13)
+    bound = 2.0 ** -8 * max(np.abs(st_o).max() for st_o, _ in cache.slots.values())
+    assert np.abs(o - full).max() <= bound * (1 + 1e-9)
+    assert np.abs(o - full).max() > 0                   # the rounding is really applied
