@@ -7,7 +7,6 @@
 
 #include <atomic>
 #include <cstring>
-#include <vector>
 
 #include "../../include/dt.h"
 #include "attn_fused.h"
@@ -194,18 +193,20 @@ extern "C" int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t
   }
   (void)d_status;
   if (stamps) {
-    // [nqt][1+m] -> [nqt][1+m2] in place, row by row (a new row never starts
-    // after its old row, and each new row is built before it is written)
-    std::vector<int32_t> tmp(1 + m2);
+    // [nqt][1+m] -> [nqt][1+m2] in place, rows and entries in increasing
+    // order with no buffer: new entry i of row qt lands at qt*(1+m2)+i, which
+    // is never after old entry i of that row, and every old entry it could
+    // cover (row < qt, or entry <= i of row qt) has already been consumed,
+    // since new entry i reads old entries factor*i+1 .. > i.
     for (int qt = 0; qt < G.nqt; ++qt) {
       const int32_t* old_row = stamps + (size_t)qt * (1 + m);
-      tmp[0] = old_row[0];
+      int32_t* new_row = stamps + (size_t)qt * (1 + m2);
+      new_row[0] = old_row[0];
       for (int i = 0; i < m2; ++i) {
         int32_t s = old_row[1 + factor * i];
         for (int j = factor * i + 1; j < factor * i + factor && j < m; ++j) s = old_row[1 + j] < s ? old_row[1 + j] : s;
-        tmp[1 + i] = s;
+        new_row[1 + i] = s;
       }
-      memcpy(stamps + (size_t)qt * (1 + m2), tmp.data(), sizeof(int32_t) * (1 + m2));
     }
   }
   if ((int64_t)p->H * p->S == 0) return DT_OK;
