@@ -37,6 +37,15 @@ notes of the repository):
     first among equal distances) and always computes {q};
   * a bf16 state cache stores OUT rounded to nearest-even bf16 and LSE in
     float64 (fp32 on the GPU);
+  * partition importance w(k) of a key set for a query tile is the normalised
+    composition weight exp(LSE_k - LSE) (the share of a row's softmax mass in
+    that set), averaged over the tile's rows and the heads, measured when all
+    sets are fresh (an anchor step); the predicted error of reusing set k is
+    ASE = w(k) * tau with tau = t - t_c its cache age (error growing linearly
+    with age at a common rate); the importance plan reuses the r sets of
+    smallest ASE, never the local set nor a never-written slot, lower index
+    first among equal values, the products taken in float32 as the GPU-side
+    weights are float32;
   * Dynamic Group State Compose by a factor k: the new group i is old groups
     k i .. k i + k - 1, its cached state their composition, its stamp the
     oldest of theirs (never written if any was never written).
@@ -58,6 +67,7 @@ MODE_PROXIMITY = 1
 MODE_ALL_REUSE = 2
 MODE_EXPLICIT = 3
 MODE_WINDOW = 4
+MODE_IMPORTANCE = 5
 
 __all__ = [
     "TILE", "REUSE", "COMPUTE", "MODE_ALL_COMPUTE", "MODE_PROXIMITY",
@@ -67,7 +77,7 @@ __all__ = [
     "proximity_row", "build_plan", "window_in", "StateCache",
     "partition_step", "window_step", "softmax_scale",
     "n_groups", "group_key_sets", "group_proximity_row", "key_sets_of_tile",
-    "compose_groups",
+    "compose_groups", "MODE_IMPORTANCE", "state_importance", "importance_row",
 ]
 
 
@@ -279,10 +289,29 @@ def key_sets_of_tile(q: int, P: int, group: int) -> List[List[int]]:
     return [[k] for k in range(P)] if group == 0 else group_key_sets(q, P, group)
 
 
+def importance_row(w_row: np.ndarray, stamps_row: np.ndarray, step: int, r: int, local: int) -> np.ndarray:
+    """[DT] error model and selection: predicted error of reusing key set k
+    is w(k) * (step - t_c(k)); the r sets with the smallest predicted error
+    are reused (lower index first among equal values).  The local set and
+    slots never written (t_c < 0) are always computed."""
+    n = len(w_row)
+    row = np.full(n, COMPUTE, dtype=np.uint8)
+    cand = []
+    for k in range(n):
+        if k == local or stamps_row[k] < 0:
+            continue
+        ase = np.float32(w_row[k]) * np.float32(step - int(stamps_row[k]))
+        cand.append((float(ase), k))
+    for _, k in sorted(cand)[:r]:
+        row[k] = REUSE
+    return row
+
+
 def build_plan(mode: int, H: int, S: int, D: int, P: int, step: int,
                r: int = 0, window: int = 0,
                stamps: Optional[np.ndarray] = None,
-               explicit: Optional[np.ndarray] = None, group: int = 0):
+               explicit: Optional[np.ndarray] = None, group: int = 0,
+               weights: Optional[np.ndarray] = None):
     """Plan, block counts, algorithmic FLOPs and updated stamps of one step.
 
     Returns ``(plan uint8 [nqt][nseg], counts, stamps')`` where nseg = P (2 in
@@ -307,6 +336,12 @@ def build_plan(mode: int, H: int, S: int, D: int, P: int, step: int,
                 plan[t] = COMPUTE
             elif mode == MODE_PROXIMITY:
                 plan[t] = proximity_row(kq, P, r) if group == 0 else group_proximity_row(kq, P, group, r)
+            elif mode == MODE_IMPORTANCE and step <= 1:
+                plan[t] = COMPUTE
+            elif mode == MODE_IMPORTANCE:
+                st_row = (np.full(nseg, -1) if stamps is None else np.asarray(stamps).reshape(nqt, nseg)[t])
+                plan[t] = importance_row(np.asarray(weights).reshape(nqt, nseg)[t], st_row, step, r,
+                                         kq if group == 0 else 0)
             elif mode == MODE_ALL_REUSE:
                 plan[t] = REUSE
             elif mode == MODE_EXPLICIT:
@@ -432,6 +467,27 @@ def partition_step(Q: np.ndarray, K: np.ndarray, V: np.ndarray, plan: np.ndarray
         for k, h_, rs, st in pending:
             cache.put(k, h_, rs, st[0], st[1])
     return O, L, fresh
+
+
+def state_importance(cache: StateCache, L: Dict[Tuple[int, int], float], S: int, P: int, group: int,
+                     heads: Sequence[int], nseg: int) -> np.ndarray:
+    """[DT] partition importance w(k) per (query tile, key set): the mean over
+    the tile's rows and the heads of exp(LSE_k - LSE), LSE_k the cached state
+    of key set k and LSE the row's final log-sum-exp (``L[(h, row)]``).  An
+    empty state or row contributes 0.  Returns float64 [nqt][nseg]."""
+    tiles = query_tiles(S, P)
+    w = np.zeros((len(tiles), nseg))
+    for t, (_, q0, q1) in enumerate(tiles):
+        for k in range(nseg):
+            tot = 0.0
+            for h in heads:
+                for row in range(q0, q1):
+                    lk = cache.slots[(k, h, row)][1]
+                    lt = L[(h, row)]
+                    if np.isfinite(lk) and np.isfinite(lt):
+                        tot += math.exp(lk - lt)
+            w[t, k] = tot / (len(heads) * (q1 - q0))
+    return w
 
 
 def _get_or_identity(cache: StateCache, k, h, rs, D):
