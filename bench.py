@@ -58,7 +58,7 @@ def parse_args():
     ap.add_argument("--group", type=int, default=0,
                     help="state grouping: groups of G adjacent partitions, --reuse then counts groups")
     ap.add_argument("--no-grouped", action="store_true",
-                    help="skip the grouped-cache, compose and bf16-cache measurements")
+                    help="skip the grouped-cache, compose, bf16-cache and importance measurements")
     return ap.parse_args()
 
 
@@ -399,8 +399,51 @@ def main():
         del graph
         return max_over_ranks([a.elapsed_time(b) / n], "cuda")[0], vc
 
-    grouped = compose = bf16c = None
+    grouped = compose = bf16c = importance = None
     if not win and grp == 0 and not args.no_grouped:
+        # importance planning: weights measured at the anchor, then the step
+        # reusing the r key sets of smallest importance x age
+        isess = Session(w.H, w.S, w.D, w.P, reuse_per_row=r)
+        isess.set_inputs(q1, k1, v1)
+        isess.step(1)
+        isess.check()
+        pimp = dt.params(w.H, w.S, w.D, w.P, dt.DT_MODE_IMPORTANCE, r, 0, 1)
+        d_w = torch.empty((isess.nqt, isess.nseg), dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            dt.dt_state_importance(pimp, isess.cache_L, isess.L, d_w, isess.status)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(cur)
+        for _ in range(10):
+            dt.dt_state_importance(pimp, isess.cache_L, isess.L, d_w, isess.status)
+        b.record(cur)
+        barrier()
+        ims = max_over_ranks([a.elapsed_time(b) / 10], "cuda")[0]
+        ibytes = (w.P + 1) * w.H * w.S * 4
+        wts = isess.measure_importance()
+        isess.mode = dt.DT_MODE_IMPORTANCE
+        isess.set_inputs(q2, k2, v2)
+        graph = isess.capture_step(2)
+        for _ in range(3):
+            graph.replay()
+        barrier()
+        a.record(cur)
+        ni = max(5, args.steps // 2)
+        for _ in range(ni):
+            ic = graph.replay()
+        b.record(cur)
+        barrier()
+        isess.check()
+        istep = max_over_ranks([a.elapsed_time(b) / ni], "cuda")[0]
+        hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        importance = {"kernel": "state_importance", "ms": ims, "bytes": ibytes,
+                      "GB/s": ibytes / (ims * 1e-3) / 1e9, "frac_of_hbm": ibytes / (ims * 1e-3) / 1e9 / hbm,
+                      "weights_row_sum_max_err": float(np.abs(wts.sum(axis=1) - 1.0).max()),
+                      "plan": f"reuse the {r} key sets of smallest importance x age per query tile",
+                      "ms_per_step": istep, "tflops": ic["computed_flops"] / (istep * 1e-3) / 1e12,
+                      "skipped_blocks": ic["skipped_blocks"], "computed_blocks": ic["computed_blocks"],
+                      "launch": "CUDA-graph replay"}
+        del graph, isess, d_w
         # the same step with the cached OUT stored in bf16
         bs = Session(w.H, w.S, w.D, w.P, reuse_per_row=r, state_dtype=dt.DT_STATE_BF16)
         bms, bc = time_session(bs)
@@ -501,6 +544,7 @@ def main():
             "grouped": grouped,
             "group_compose": compose,
             "bf16_state_cache": bf16c,
+            "importance": importance,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -68,6 +68,9 @@ extern "C" {
 #define DT_MODE_ALL_REUSE   2  /* every pair reused */
 #define DT_MODE_EXPLICIT    3  /* plan copied from the caller */
 #define DT_MODE_WINDOW      4  /* window + residual: 2 key sets per query tile */
+#define DT_MODE_IMPORTANCE  5  /* step 1: anchor; later steps: the r key sets of smallest
+                                  predicted error (importance x cache age) are reused;
+                                  built by dt_plan_build_importance */
 
 #define DT_PLAN_REUSE   0
 #define DT_PLAN_COMPUTE 1
@@ -133,6 +136,19 @@ DT_API int dt_plan_geometry(const dt_plan_params* p, int32_t* nqt, int32_t* nseg
  * untouched), then sets stamp = step on COMPUTE entries and fills the counts.
  * Host only, no CUDA call.  Errors: DT_ERR_INVALID, DT_ERR_CACHE_EMPTY. */
 DT_API int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, dt_plan* out);
+
+/* Importance plan of one step ("DiTango", error model and selection
+ * strategy: the error of reusing a cached state is its partition importance
+ * times a growth over cache age).  p->mode must be DT_MODE_IMPORTANCE (either
+ * key-set layout).  weights: host float [nqt][nseg], the importance of each
+ * key set for each query tile (dt_state_importance, measured at an anchor).
+ * Step 1 computes everything.  Later steps, per query tile: predicted error
+ * e_k = weights[k] * (step - stamp_k), a float product; the local key set
+ * (partition q, or set 0 when grouped) and slots with stamp < 0 are never
+ * reused; the r = p->reuse_per_row sets of smallest e_k are reused, the lower
+ * index first among equal values (fewer if fewer are eligible).  Then stamps
+ * and counts as dt_plan_build.  Host only.  Errors: DT_ERR_INVALID. */
+DT_API int dt_plan_build_importance(const dt_plan_params* p, const float* weights, dt_plan* out);
 
 /* Fused step on the GPU ("DiTango", attention state Eq. 1-3, composition Eq. 4,
  * selective reuse Fig. 6).  For each head and query tile and each key set of
@@ -212,6 +228,18 @@ DT_API int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_plan,
  * null cache), DT_ERR_UNSUPPORTED (misaligned cache pointers, bf16 states). */
 DT_API int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t* stamps,
                      float* cache_O, float* cache_L, int32_t* d_status, void* stream);
+
+/* Partition importance ("DiTango", error model: the normalised composition
+ * weight of a state, Eq. 4): weights[qt][k] = mean over the query tile's rows
+ * and all heads of exp(cache_L[k][h][row] - L[h][row]), the share of each
+ * row's softmax mass that falls on key set k (0 where either LSE is -inf).
+ * Meaningful after a step that computed every key set (an anchor), whose
+ * outputs are L and whose fresh states are in cache_L.  Partition modes
+ * (either layout).  cache_L fp32 [nseg][H][S], L fp32 [H][S] (read),
+ * d_weights fp32 [nqt][nseg] (device, written).  One launch, HBM-bound.
+ * Errors: DT_ERR_INVALID, DT_ERR_UNSUPPORTED (misaligned pointers). */
+DT_API int dt_state_importance(const dt_plan_params* p, const float* cache_L, const float* L,
+                        float* d_weights, int32_t* d_status, void* stream);
 
 #define DT_WR_MAKE  0   /* R = O_full - O_win                 */
 #define DT_WR_APPLY 1   /* O = bf16(O_win + R)  (O_full unused) */

@@ -24,10 +24,12 @@ __all__ = [
     "DT_OK", "DT_ERR_INVALID", "DT_ERR_UNSUPPORTED", "DT_ERR_CACHE_EMPTY", "DT_ERR_CUDA",
     "DT_ERR_TIMEOUT", "DT_MODE_ALL_COMPUTE", "DT_MODE_PROXIMITY", "DT_MODE_ALL_REUSE",
     "DT_MODE_EXPLICIT", "DT_MODE_WINDOW", "DT_PLAN_REUSE", "DT_PLAN_COMPUTE", "DT_WR_MAKE",
-    "DT_WR_APPLY", "DT_TILE", "DT_STATE_F32", "DT_STATE_BF16",
+    "DT_WR_APPLY", "DT_TILE", "DT_STATE_F32", "DT_STATE_BF16", "DT_MODE_IMPORTANCE",
+    "dt_plan_build_importance", "dt_state_importance",
 ]
 
 DT_OK, DT_ERR_INVALID, DT_ERR_UNSUPPORTED, DT_ERR_CACHE_EMPTY, DT_ERR_CUDA, DT_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+DT_MODE_IMPORTANCE = 5
 DT_STATE_F32, DT_STATE_BF16 = 0, 1
 DT_MODE_ALL_COMPUTE, DT_MODE_PROXIMITY, DT_MODE_ALL_REUSE, DT_MODE_EXPLICIT, DT_MODE_WINDOW = 0, 1, 2, 3, 4
 DT_PLAN_REUSE, DT_PLAN_COMPUTE = 0, 1
@@ -81,6 +83,8 @@ def load() -> ctypes.CDLL:
             "dt_state_cache_update": ([pp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_window_residual": ([i32, i32, i32, i32, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_group_compose": ([pp, i32, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_plan_build_importance": ([pp, vp, ctypes.POINTER(Plan)], ctypes.c_int),
+            "dt_state_importance": ([pp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_set_wait_limit_ns": ([i64], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -142,6 +146,31 @@ def dt_plan_build(p: PlanParams, stamps: Optional[np.ndarray] = None, explicit: 
     _check(load().dt_plan_build(ctypes.byref(p), _ptr(ex), ctypes.byref(out)), "dt_plan_build")
     return plan, {"computed_blocks": out.computed_blocks, "skipped_blocks": out.skipped_blocks,
                   "computed_flops": out.computed_flops}
+
+
+def dt_plan_build_importance(p: PlanParams, weights: Optional[np.ndarray], stamps: Optional[np.ndarray] = None):
+    """Importance plan of one step (p.mode = DT_MODE_IMPORTANCE).  weights:
+    float32 [nqt][nseg] (host).  Returns (plan, counts) like dt_plan_build;
+    ``stamps`` is updated in place when given."""
+    nqt, nseg = dt_plan_geometry(p)
+    plan = np.zeros((nqt, nseg), dtype=np.uint8)
+    out = Plan()
+    out.plan = plan.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+    if stamps is not None:
+        assert stamps.dtype == np.int32 and stamps.flags.c_contiguous and stamps.size == nqt * nseg
+        out.stamps = stamps.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    w = None
+    if weights is not None:
+        w = np.ascontiguousarray(weights, dtype=np.float32)
+        assert w.size == nqt * nseg
+    _check(load().dt_plan_build_importance(ctypes.byref(p), _ptr(w), ctypes.byref(out)), "dt_plan_build_importance")
+    return plan, {"computed_blocks": out.computed_blocks, "skipped_blocks": out.skipped_blocks,
+                  "computed_flops": out.computed_flops}
+
+
+def dt_state_importance(p: PlanParams, cache_L, L, d_weights, d_status=None, stream=None) -> None:
+    _check(load().dt_state_importance(ctypes.byref(p), _ptr(cache_L), _ptr(L), _ptr(d_weights), _ptr(d_status),
+                                      _stream(stream)), "dt_state_importance")
 
 
 def dt_attn_partial_fused(p: PlanParams, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,

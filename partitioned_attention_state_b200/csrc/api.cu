@@ -78,7 +78,7 @@ extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head
                                            const uint8_t* d_plan, const void* Q, const void* K, const void* V,
                                            float* cache_O, float* cache_L, float* R, void* O, float* L,
                                            int64_t* d_counters, int32_t* d_status, void* stream) {
-  if (!p || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW) return DT_ERR_INVALID;
+  if (!p || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE) return DT_ERR_INVALID;
   const bool win = p->mode == DT_MODE_WINDOW;
   if (!shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (win ? p->window < 1 : p->P < 1) return DT_ERR_INVALID;
@@ -161,7 +161,7 @@ extern "C" int dt_state_merge(int32_t N, int32_t H, int32_t S, int32_t D, const 
 extern "C" int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_plan, const float* fresh_O,
                                      const float* fresh_L, float* cache_O, float* cache_L, int32_t* d_status,
                                      void* stream) {
-  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW)
+  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE)
     return DT_ERR_INVALID;
   if (p->P < 1 || p->group < 0 || p->D < 4 || p->D % 4 != 0 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (p->state_dtype != DT_STATE_F32) return DT_ERR_UNSUPPORTED;
@@ -179,7 +179,7 @@ extern "C" int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_p
 
 extern "C" int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t* stamps, float* cache_O,
                                 float* cache_L, int32_t* d_status, void* stream) {
-  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW)
+  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE)
     return DT_ERR_INVALID;
   if (p->P < 1 || p->group < 1 || factor < 2 || factor > 8) return DT_ERR_INVALID;
   if (p->state_dtype != DT_STATE_F32) return DT_ERR_UNSUPPORTED;
@@ -214,6 +214,21 @@ extern "C" int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t
   if (int e = sm_count(&sms)) return e;
   return dt::launch_group_compose(m, factor, p->H, p->S, p->D, cache_O, cache_L, sms,
                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int dt_state_importance(const dt_plan_params* p, const float* cache_L, const float* L, float* d_weights,
+                                   int32_t* d_status, void* stream) {
+  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE)
+    return DT_ERR_INVALID;
+  if (p->P < 1 || p->group < 0 || p->D < 1 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
+  const dt::Geom G = dt::make_geom(p->H, p->S, p->D, p->P, 0, p->group);
+  if ((int64_t)G.nqt * G.P == 0) return DT_OK;
+  if (!d_weights) return DT_ERR_INVALID;
+  if (p->H == 0) return dt::launch_fill_zero(d_weights, (int64_t)G.nqt * G.P, reinterpret_cast<cudaStream_t>(stream));
+  if (!cache_L || !L) return DT_ERR_INVALID;
+  if (!aligned16(cache_L) || !aligned16(L) || !aligned16(d_weights)) return DT_ERR_UNSUPPORTED;
+  (void)d_status;
+  return dt::launch_state_importance(G, cache_L, L, d_weights, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int dt_window_residual(int32_t op, int32_t H, int32_t S, int32_t D, const float* O_full,

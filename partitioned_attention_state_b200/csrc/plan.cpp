@@ -20,14 +20,16 @@ namespace {
 bool params_ok(const dt_plan_params* p) {
   if (!p) return false;
   if (p->H < 0 || p->S < 0 || p->D < 1 || p->step < 1) return false;
-  if (p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_WINDOW) return false;
+  if (p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE) return false;
   if (p->group < 0) return false;
   if (p->mode == DT_MODE_WINDOW) {
     if (p->window < 1 || p->group != 0) return false;
   } else {
     if (p->P < 1) return false;
     const int rmax = p->group > 0 ? dt::ceil_div(p->P, p->group) : p->P - 1;
-    if (p->mode == DT_MODE_PROXIMITY && (p->reuse_per_row < 0 || p->reuse_per_row > rmax)) return false;
+    if ((p->mode == DT_MODE_PROXIMITY || p->mode == DT_MODE_IMPORTANCE) &&
+        (p->reuse_per_row < 0 || p->reuse_per_row > rmax))
+      return false;
   }
   return true;
 }
@@ -105,8 +107,13 @@ extern "C" int dt_plan_geometry(const dt_plan_params* p, int32_t* nqt, int32_t* 
   return DT_OK;
 }
 
+namespace {
+int finish_plan(const dt_plan_params* p, const dt::Geom& g, dt_plan* out);
+}
+
 extern "C" int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, dt_plan* out) {
   if (!params_ok(p) || !out || !out->plan) return DT_ERR_INVALID;
+  if (p->mode == DT_MODE_IMPORTANCE) return DT_ERR_INVALID;       // needs weights
   dt::Geom g = geom_of(p);
   const int nqt = g.nqt, nseg = g.P;
   out->nqt = nqt;
@@ -143,7 +150,47 @@ extern "C" int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_pl
         break;
     }
   }
+  return finish_plan(p, g, out);
+}
 
+extern "C" int dt_plan_build_importance(const dt_plan_params* p, const float* weights, dt_plan* out) {
+  if (!params_ok(p) || !out || !out->plan || p->mode != DT_MODE_IMPORTANCE) return DT_ERR_INVALID;
+  dt::Geom g = geom_of(p);
+  const int nqt = g.nqt, nseg = g.P;
+  if (!weights && p->step > 1 && nqt > 0) return DT_ERR_INVALID;
+  out->nqt = nqt;
+  out->nseg = nseg;
+  out->computed_blocks = out->skipped_blocks = out->computed_flops = 0;
+  for (int qt = 0; qt < nqt; ++qt) {
+    uint8_t* row = out->plan + (size_t)qt * nseg;
+    for (int k = 0; k < nseg; ++k) row[k] = DT_PLAN_COMPUTE;
+    if (p->step <= 1) continue;                                   // anchor
+    const int local = g.grp > 0 ? 0 : dt::query_tile<0>(g, qt).part;
+    const float* w = weights + (size_t)qt * nseg;
+    const int32_t* st = out->stamps ? out->stamps + (size_t)qt * nseg : nullptr;
+    // r times: the eligible set of smallest predicted error, lower index on ties
+    for (int taken = 0; taken < p->reuse_per_row; ++taken) {
+      int best = -1;
+      float best_e = 0.f;
+      for (int k = 0; k < nseg; ++k) {
+        if (k == local || row[k] == DT_PLAN_REUSE || !st || st[k] < 0) continue;
+        const float e = w[k] * (float)(p->step - st[k]);
+        if (best < 0 || e < best_e) { best = k; best_e = e; }
+      }
+      if (best < 0) break;
+      row[best] = DT_PLAN_REUSE;
+    }
+  }
+  return finish_plan(p, g, out);
+}
+
+namespace {
+
+// Shared tail of the plan builders: refuse REUSE of never-written slots,
+// stamp the COMPUTE slots, fill the counts.
+int finish_plan(const dt_plan_params* p, const dt::Geom& g, dt_plan* out) {
+  const int nqt = g.nqt, nseg = g.P;
+  uint8_t* plan = out->plan;
   // validate reuse against stamps before touching them
   const size_t n = (size_t)nqt * nseg;
   for (size_t i = 0; i < n; ++i) {
@@ -191,3 +238,5 @@ extern "C" int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_pl
   out->computed_flops = fl;
   return DT_OK;
 }
+
+}  // namespace

@@ -1,6 +1,6 @@
 // state_ops.cu -- HBM-bound state kernels of libdt: N-way state composition,
-// plan-driven cache scatter, in-place regrouping of cached group states, and
-// the window residual (make / apply).
+// plan-driven cache scatter, in-place regrouping of cached group states,
+// partition importance, and the window residual (make / apply).
 //
 // All three stream rows of D fp32 values with 16-byte vector accesses over a
 // flat index, so consecutive threads touch consecutive 16-byte words (fully
@@ -168,6 +168,38 @@ __global__ void __launch_bounds__(kBlock) group_compose_kernel(int m, int factor
   }
 }
 
+// "DiTango", partition importance: the normalised composition weight
+// exp(LSE_k - LSE) of key set k for each row, averaged over the rows of a
+// query tile and the heads.  One block per (query tile, key set).
+__global__ void __launch_bounds__(kBlock) state_importance_kernel(Geom G, const float* __restrict__ cL,
+                                                                  const float* __restrict__ L,
+                                                                  float* __restrict__ w) {
+  __shared__ float part[kBlock / 32];
+  const int qt = blockIdx.x / G.P, k = blockIdx.x - qt * G.P;
+  const QTile t = query_tile<kModePartition>(G, qt);
+  const int n = G.H * t.rows;
+  float acc = 0.f;
+  for (int i = threadIdx.x; i < n; i += kBlock) {
+    const int h = i / t.rows, r = t.q0 + (i - h * t.rows);
+    const float lk = cL[((int64_t)k * G.H + h) * G.S + r], lt = L[(int64_t)h * G.S + r];
+    if (lk > kNegInf && lt > kNegInf) acc += expf(lk - lt);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int j = 0; j < kBlock / 32; ++j) tot += part[j];
+    w[blockIdx.x] = n > 0 ? tot / (float)n : 0.f;
+  }
+}
+
+__global__ void __launch_bounds__(kBlock) fill_zero_kernel(float* __restrict__ x, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    x[i] = 0.f;
+}
+
 int grid_for(int64_t work, int sms) {
   int64_t blocks = (work + kBlock - 1) / kBlock;
   int64_t cap = (int64_t)sms * 8;           // 8 resident 256-thread blocks per SM
@@ -201,6 +233,17 @@ int launch_group_compose(int m, int factor, int H, int S, int D, float* cO, floa
     case 4: group_compose_kernel<4><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL); break;
     default: group_compose_kernel<8><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL); break;   // 5..8
   }
+  return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+}
+
+int launch_state_importance(const Geom& G, const float* cL, const float* L, float* w, cudaStream_t st) {
+  const int64_t blocks = (int64_t)G.nqt * G.P;
+  state_importance_kernel<<<(unsigned)blocks, kBlock, 0, st>>>(G, cL, L, w);
+  return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+}
+
+int launch_fill_zero(float* x, int64_t n, cudaStream_t st) {
+  fill_zero_kernel<<<(unsigned)((n + kBlock - 1) / kBlock < 1024 ? (n + kBlock - 1) / kBlock : 1024), kBlock, 0, st>>>(x, n);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
 }
 

@@ -13,6 +13,8 @@ int launch_state_merge(int N, int H, int S, int D, const float* O_in, const floa
 int launch_cache_update(const Geom& G, const uint8_t* plan, const float* fO, const float* fL, float* cO, float* cL,
                         int sms, cudaStream_t st);
 int launch_group_compose(int m, int factor, int H, int S, int D, float* cO, float* cL, int sms, cudaStream_t st);
+int launch_state_importance(const Geom& G, const float* cL, const float* L, float* w, cudaStream_t st);
+int launch_fill_zero(float* x, int64_t n, cudaStream_t st);
 int launch_window_residual(int op, int64_t n, const float* Of, const float* Ow, float* R, void* O, int sms,
                            cudaStream_t st);
 

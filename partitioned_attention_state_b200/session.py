@@ -16,8 +16,9 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused, dt_attn_partial_fused_heads, dt_group_compose,
-               dt_plan_build, dt_plan_geometry, DtError, params)
+from . import (DT_MODE_IMPORTANCE, DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused,
+               dt_attn_partial_fused_heads, dt_group_compose, dt_plan_build, dt_plan_build_importance, dt_plan_geometry,
+               dt_state_importance, DtError, params)
 
 
 def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
@@ -61,6 +62,7 @@ class Session:
         self.counters = torch.zeros(4, dtype=torch.int64, device=dev)
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
         self.stamps = np.full((self.nqt, self.nseg), -1, dtype=np.int32)
+        self.weights: Optional[np.ndarray] = None
         self.last_counts = None
         self.last_plan = None
 
@@ -107,8 +109,25 @@ class Session:
         win = mode == DT_MODE_WINDOW
         p = params(self.H, self.S, self.D, 1 if win else self.P, mode, self.r, self.window, step,
                    0 if win else self.group, 0 if win else self.state_dtype)
-        plan, counts = dt_plan_build(p, self.stamps, explicit)
+        if mode == DT_MODE_IMPORTANCE:
+            plan, counts = dt_plan_build_importance(p, self.weights, self.stamps)
+        else:
+            plan, counts = dt_plan_build(p, self.stamps, explicit)
         return p, plan, counts
+
+    def measure_importance(self) -> np.ndarray:
+        """Partition importance of every (query tile, key set) from the cached
+        LSEs and the last step's L (dt_state_importance).  Call it after a
+        step that computed every key set (an anchor); later steps in
+        DT_MODE_IMPORTANCE plan with it.  Synchronises; returns the float32
+        weights [nqt][nseg] kept in ``self.weights``."""
+        if self.cache_L is None or self.mode == DT_MODE_WINDOW:
+            raise ValueError("importance needs a partition-mode session with a cache")
+        p = params(self.H, self.S, self.D, self.P, DT_MODE_IMPORTANCE, self.r, 0, 1, self.group, self.state_dtype)
+        d_w = torch.empty((max(self.nqt, 1), self.nseg), dtype=torch.float32, device=self.device)
+        dt_state_importance(p, self.cache_L, self.L, d_w, self.status)
+        self.weights = d_w[: self.nqt].cpu().numpy().copy()
+        return self.weights
 
     # -------------------------------------------------------------- one step
     def step(self, step: int, mode: Optional[int] = None, explicit: Optional[np.ndarray] = None,

@@ -265,3 +265,51 @@ def test_state_dtype_validated():
     a, ca = dt.dt_plan_build(dt.params(1, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1), None)
     b, cb = dt.dt_plan_build(dt.params(1, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1, 0, dt.DT_STATE_BF16), None)
     assert np.array_equal(a, b) and ca == cb
+
+
+@pytest.mark.parametrize("S,P,g", [(1024, 4, 0), (2600, 7, 0), (32760, 16, 4), (1800, 12, 5), (640, 8, 1)])
+def test_importance_plan_matches_oracle(S, P, g):
+    """dt_plan_build_importance against the oracle's rule, bit for bit, on
+    random weights with exact ties and random stamps (never-written slots
+    included), through steps 1-3."""
+    H, D = 2, 64
+    p = dt.params(H, S, D, P, dt.DT_MODE_IMPORTANCE, 2, 0, 1, g)
+    nqt, nseg = dt.dt_plan_geometry(p)
+    rng = np.random.default_rng(S + P + g)
+    w = rng.random((nqt, nseg)).astype(np.float32)
+    w[::3] = np.round(w[::3] * 4) / 4                       # exact ties
+    for r in (0, 1, 2, nseg - 1):
+        st = rng.integers(-1, 3, size=(nqt, nseg)).astype(np.int32)
+        st_o = st.copy()
+        for step in (1, 2, 3):
+            p = dt.params(H, S, D, P, dt.DT_MODE_IMPORTANCE, r, 0, step, g)
+            plan_c, counts_c = dt.dt_plan_build_importance(p, w, st)
+            plan_o, counts_o, st_o = orc.build_plan(orc.MODE_IMPORTANCE, H, S, D, P, step, r=r, stamps=st_o,
+                                                    group=g, weights=w)
+            np.testing.assert_array_equal(plan_c, plan_o)
+            assert counts_c == counts_o
+            np.testing.assert_array_equal(st, st_o)
+
+
+def test_importance_calls_validated():
+    import ctypes
+    lib = dt.load()
+    p = dt.params(1, 1024, 64, 4, dt.DT_MODE_IMPORTANCE, 1, 0, 2)
+    nqt, nseg = dt.dt_plan_geometry(p)
+    plan = np.zeros((nqt, nseg), np.uint8)
+    out = dt.Plan()
+    out.plan = plan.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+    assert lib.dt_plan_build(ctypes.byref(p), None, ctypes.byref(out)) == dt.DT_ERR_INVALID       # needs weights
+    assert lib.dt_plan_build_importance(ctypes.byref(p), None, ctypes.byref(out)) == dt.DT_ERR_INVALID
+    p.step = 1                                                                                        # anchor: no weights needed
+    assert lib.dt_plan_build_importance(ctypes.byref(p), None, ctypes.byref(out)) == dt.DT_OK and plan.all()
+    pp = dt.params(1, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 2)
+    w = np.ones((nqt, nseg), np.float32)
+    assert lib.dt_plan_build_importance(ctypes.byref(pp), w.ctypes.data, ctypes.byref(out)) == dt.DT_ERR_INVALID
+    p.reuse_per_row, p.step = 4, 2                                                                    # r > P - 1
+    assert lib.dt_plan_build_importance(ctypes.byref(p), w.ctypes.data, ctypes.byref(out)) == dt.DT_ERR_INVALID
+    pw = dt.params(1, 1024, 64, 1, dt.DT_MODE_WINDOW, 0, 64, 1)
+    assert lib.dt_state_importance(ctypes.byref(pw), None, None, None, None, None) == dt.DT_ERR_INVALID
+    assert lib.dt_state_importance(ctypes.byref(pp), None, None, None, None, None) == dt.DT_ERR_INVALID
+    assert lib.dt_state_importance(ctypes.byref(pp), 16 * 1024, 16 * 1024, 16 * 1024 + 4, None, None) == \
+        dt.DT_ERR_UNSUPPORTED

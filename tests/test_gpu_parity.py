@@ -400,3 +400,34 @@ def test_bf16_state_cache_video_full_size_sampled_rows():
     sched = [(1, dt.DT_MODE_PROXIMITY, 8, None), (2, dt.DT_MODE_PROXIMITY, 8, None)]
     run_partition_schedule(w.H, w.S, w.D, w.P, sched, wl.stream_for(w).next_step, heads=[0, 39],
                            rows=sample_rows(w.S, w.P, n_extra=16), state_dtype=dt.DT_STATE_BF16)
+
+
+# ------------------------------------------------------ partition importance
+
+@pytest.mark.parametrize("H,S,D,P,g", [(2, 1024, 64, 4, 0), (2, 2048, 128, 16, 4), (3, 1800, 72, 12, 5),
+                                       (2, 2600, 64, 7, 0)])
+def test_importance_weights_and_plan_match_oracle(H, S, D, P, g):
+    """dt_state_importance after an anchor equals the oracle's importance of
+    the same inputs, the weights of a row sum to one, and importance-planned
+    steps use the oracle's rule on those weights and match it in output."""
+    s = wl.InputStream(H, S, D, 0.05, seed=S + P)
+    inputs = [s.next_step() for _ in range(3)]
+    it = iter(inputs)
+    sess, cache = run_partition_schedule(H, S, D, P, [(1, dt.DT_MODE_PROXIMITY, 0, None)], lambda: next(it),
+                                         group=g)
+    w_gpu = sess.measure_importance()
+    assert w_gpu.shape == (sess.nqt, sess.nseg) and w_gpu.dtype == np.float32
+    np.testing.assert_allclose(w_gpu.sum(axis=1), 1.0, rtol=0, atol=1e-4)
+    q, k, v = inputs[0]
+    oc = orc.StateCache()
+    plan1, _, _ = orc.build_plan(orc.MODE_ALL_COMPUTE, H, S, D, P, step=1, group=g)
+    _, L, _ = orc.partition_step(q, k, v, plan1, S, P, oc, group=g)
+    Lmap = {(h, r): float(L[h, r]) for h in range(H) for r in range(S)}
+    w_ref = orc.state_importance(oc, Lmap, S, P, g, range(H), sess.nseg)
+    np.testing.assert_allclose(w_gpu, w_ref, rtol=0, atol=2e-3)
+    for step in (2, 3):
+        want, _, _ = orc.build_plan(orc.MODE_IMPORTANCE, H, S, D, P, step, r=2, stamps=sess.stamps.copy(), group=g,
+                                    weights=w_gpu)
+        run_partition_schedule(H, S, D, P, [(step, dt.DT_MODE_IMPORTANCE, 2, None)], lambda: next(it),
+                               check_untouched=True, sess=sess, cache=cache)
+        np.testing.assert_array_equal(sess.last_plan, want)
