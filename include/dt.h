@@ -6,12 +6,16 @@
  * per-step plan either COMPUTEs a fresh partial attention state or REUSEs the
  * state of that pair cached at an earlier step; the output is the
  * log-sum-exp weighted composition of all P states, and fresh states
- * overwrite their cache slots.  Window attention with a cached
- * full-minus-window residual is a second plan mode on the same machinery.
+ * overwrite their cache slots.  Partitions can be grouped (one composed
+ * state per group of adjacent partitions), cached states regrouped in place,
+ * stored with a bf16 OUT, and plans ranked by measured partition importance
+ * and cache age.  Window attention with a cached full-minus-window residual
+ * is a further plan mode on the same machinery.
  *
  * Sources: "DiTango: Cost-Effective Parallel Diffusion Generation with
  * Selective Attention State Reuse" (attention state, Eq. 1-3; composition,
- * Eq. 4; selective compute and reuse, Fig. 6; anchor steps) and
+ * Eq. 4; selective compute and reuse, Fig. 6; anchor steps; state grouping
+ * and Dynamic Group State Compose; error model and selection strategy) and
  * "DiTFastAttn: Attention Compression for Diffusion Transformer Models"
  * (summary page, Approach: window attention with residual sharing).
  *
@@ -28,7 +32,8 @@
  *   - tensors are dense, row-major, batch 1:
  *       Q, K, V, O           bf16  [H][S][D]
  *       L (final LSE)        fp32  [H][S]
- *       cache_O              fp32  [nseg][H][S][D] (state OUT of key set k)
+ *       cache_O              fp32  [nseg][H][S][D] (state OUT of key set k;
+ *                                   bf16 with state_dtype = DT_STATE_BF16)
  *       cache_L              fp32  [nseg][H][S]    (state LSE of key set k)
  *       R (window residual)  fp32  [H][S][D]
  *     The state of query row s, head h, key set k (KV partition k, or the
@@ -55,7 +60,9 @@ extern "C" {
 /* ---- status codes -------------------------------------------------------- */
 #define DT_OK               0
 #define DT_ERR_INVALID     -1  /* bad argument: shape, null pointer, mode, plan value */
-#define DT_ERR_UNSUPPORTED -2  /* D not in {64, 72, 128}, or a misaligned pointer */
+#define DT_ERR_UNSUPPORTED -2  /* D not in {64, 72, 128}, a misaligned pointer, more than 64
+                                  key sets in the fused step, or a bf16 state cache given to a
+                                  call that takes fp32 states only */
 #define DT_ERR_CACHE_EMPTY -3  /* a REUSE entry names a slot never written (stamp < 0) */
 #define DT_ERR_CUDA        -4  /* a CUDA runtime/driver call failed */
 #define DT_ERR_TIMEOUT     -5  /* (device) a bounded wait inside a kernel ran out */
