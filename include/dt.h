@@ -259,6 +259,16 @@ DT_API int dt_window_residual(int32_t op, int32_t H, int32_t S, int32_t D,
                        const float* O_full, const float* O_win,
                        float* R, void* O, int32_t* d_status, void* stream);
 
+/* Attention sharing ("DiTFastAttn", attention sharing across CFG branches
+ * and across timesteps: a branch or step takes another's attention output
+ * instead of computing its own): copies the outputs of n_heads heads,
+ * O bf16 [n_heads][S][D] and L fp32 [n_heads][S], from src to dst on the
+ * stream (device memory; src and dst ranges must not overlap unless equal,
+ * in which case nothing is done).  Errors: DT_ERR_INVALID (negative sizes,
+ * null or partially overlapping buffers), DT_ERR_CUDA. */
+DT_API int dt_share_output(int32_t n_heads, int32_t S, int32_t D, const void* src_O, const float* src_L,
+                    void* dst_O, float* dst_L, void* stream);
+
 /* Limit, in nanoseconds, of every bounded wait inside the fused kernel
  * (default 2e9).  A wait that runs out writes DT_ERR_TIMEOUT to *d_status and
  * the kernel drains its in-flight copies, frees its tensor memory and

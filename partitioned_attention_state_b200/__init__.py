@@ -25,7 +25,7 @@ __all__ = [
     "DT_ERR_TIMEOUT", "DT_MODE_ALL_COMPUTE", "DT_MODE_PROXIMITY", "DT_MODE_ALL_REUSE",
     "DT_MODE_EXPLICIT", "DT_MODE_WINDOW", "DT_PLAN_REUSE", "DT_PLAN_COMPUTE", "DT_WR_MAKE",
     "DT_WR_APPLY", "DT_TILE", "DT_STATE_F32", "DT_STATE_BF16", "DT_MODE_IMPORTANCE",
-    "dt_plan_build_importance", "dt_state_importance",
+    "dt_plan_build_importance", "dt_state_importance", "dt_share_output",
 ]
 
 DT_OK, DT_ERR_INVALID, DT_ERR_UNSUPPORTED, DT_ERR_CACHE_EMPTY, DT_ERR_CUDA, DT_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
@@ -85,6 +85,7 @@ def load() -> ctypes.CDLL:
             "dt_group_compose": ([pp, i32, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_plan_build_importance": ([pp, vp, ctypes.POINTER(Plan)], ctypes.c_int),
             "dt_state_importance": ([pp, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_share_output": ([i32, i32, i32, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_set_wait_limit_ns": ([i64], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -171,6 +172,11 @@ def dt_plan_build_importance(p: PlanParams, weights: Optional[np.ndarray], stamp
 def dt_state_importance(p: PlanParams, cache_L, L, d_weights, d_status=None, stream=None) -> None:
     _check(load().dt_state_importance(ctypes.byref(p), _ptr(cache_L), _ptr(L), _ptr(d_weights), _ptr(d_status),
                                       _stream(stream)), "dt_state_importance")
+
+
+def dt_share_output(n_heads: int, S: int, D: int, src_O, src_L, dst_O, dst_L, stream=None) -> None:
+    _check(load().dt_share_output(n_heads, S, D, _ptr(src_O), _ptr(src_L), _ptr(dst_O), _ptr(dst_L),
+                                  _stream(stream)), "dt_share_output")
 
 
 def dt_attn_partial_fused(p: PlanParams, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,

@@ -231,6 +231,27 @@ extern "C" int dt_state_importance(const dt_plan_params* p, const float* cache_L
   return dt::launch_state_importance(G, cache_L, L, d_weights, reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace {
+bool overlap(const void* a, const void* b, size_t n) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + n && y < x + n;
+}
+}  // namespace
+
+extern "C" int dt_share_output(int32_t n_heads, int32_t S, int32_t D, const void* src_O, const float* src_L,
+                               void* dst_O, float* dst_L, void* stream) {
+  if (n_heads < 0 || S < 0 || D < 1 || !shape_ok(n_heads, S, D)) return DT_ERR_INVALID;
+  const size_t nO = (size_t)n_heads * S * D * 2, nL = (size_t)n_heads * S * 4;
+  if (nO == 0) return DT_OK;
+  if (!src_O || !src_L || !dst_O || !dst_L) return DT_ERR_INVALID;
+  const bool sameO = src_O == dst_O, sameL = src_L == dst_L;
+  if ((!sameO && overlap(src_O, dst_O, nO)) || (!sameL && overlap(src_L, dst_L, nL))) return DT_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!sameO && cudaMemcpyAsync(dst_O, src_O, nO, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return DT_ERR_CUDA;
+  if (!sameL && cudaMemcpyAsync(dst_L, src_L, nL, cudaMemcpyDeviceToDevice, st) != cudaSuccess) return DT_ERR_CUDA;
+  return DT_OK;
+}
+
 extern "C" int dt_window_residual(int32_t op, int32_t H, int32_t S, int32_t D, const float* O_full,
                                   const float* O_win, float* R, void* O, int32_t* d_status, void* stream) {
   if (op != DT_WR_MAKE && op != DT_WR_APPLY) return DT_ERR_INVALID;

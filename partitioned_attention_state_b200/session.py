@@ -18,7 +18,7 @@ import torch
 
 from . import (DT_MODE_IMPORTANCE, DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused,
                dt_attn_partial_fused_heads, dt_group_compose, dt_plan_build, dt_plan_build_importance, dt_plan_geometry,
-               dt_state_importance, DtError, params)
+               dt_share_output, dt_state_importance, DtError, params)
 
 
 def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
@@ -211,6 +211,46 @@ class Session:
             cur.wait_stream(st)
         self.last_counts, self.last_plan = counts, plan
         return counts
+
+    def step_cfg_shared(self, step: int, mode: Optional[int] = None, explicit: Optional[np.ndarray] = None,
+                        stream=None) -> dict:
+        """Attention sharing across CFG branches: the session's H heads are the
+        conditional half [0, H/2) and the unconditional half [H/2, H) of one
+        layer.  Only the conditional half is computed (plan, cache slots and
+        stamps as in step()); its O and L are then copied to the unconditional
+        half, whose inputs are not read and whose cache slots stay untouched.
+        Returns the counts of the whole batch, the unconditional half's blocks
+        counted as skipped."""
+        if self.H % 2:
+            raise ValueError("CFG sharing needs an even number of heads (two branches)")
+        hb = self.H // 2
+        p, plan, counts = self.plan(step, mode, explicit)
+        st = torch.cuda.current_stream(self.device) if stream is None else stream
+        self._upload_plan(plan, st)
+        dt_attn_partial_fused_heads(p, 0, hb, self.d_plan, self.Q, self.K, self.V, self.cache_O, self.cache_L,
+                                    self.R, self.O, self.L, self.counters, self.status, st)
+        dt_share_output(hb, self.S, self.D, self.O[:hb], self.L[:hb], self.O[hb:], self.L[hb:], st)
+        total = counts["computed_blocks"] + counts["skipped_blocks"]
+        out = {"computed_blocks": counts["computed_blocks"] // 2,
+               "skipped_blocks": total - counts["computed_blocks"] // 2,
+               "computed_flops": counts["computed_flops"] // 2}
+        self.last_counts, self.last_plan = out, plan
+        return out
+
+    def share_previous_output(self) -> dict:
+        """Attention sharing across timesteps: this step takes the previous
+        step's attention output, which O and L already hold.  Nothing is
+        launched; plan, cache and stamps are untouched.  Returns the counts
+        (every block skipped, no FLOPs)."""
+        win = self.mode == DT_MODE_WINDOW
+        p = params(self.H, self.S, self.D, 1 if win else self.P, 0, 0, self.window, 1, 0 if win else self.group)
+        if win:
+            p.mode = DT_MODE_WINDOW
+        _, full = dt_plan_build(p, None)
+        out = {"computed_blocks": 0, "skipped_blocks": full["computed_blocks"] + full["skipped_blocks"],
+               "computed_flops": 0}
+        self.last_counts = out
+        return out
 
     def launch(self, p, stream=None) -> None:
         dt_attn_partial_fused(p, self.d_plan, self.Q, self.K, self.V, self.cache_O, self.cache_L, self.R, self.O,

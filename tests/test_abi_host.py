@@ -313,3 +313,15 @@ def test_importance_calls_validated():
     assert lib.dt_state_importance(ctypes.byref(pp), None, None, None, None, None) == dt.DT_ERR_INVALID
     assert lib.dt_state_importance(ctypes.byref(pp), 16 * 1024, 16 * 1024, 16 * 1024 + 4, None, None) == \
         dt.DT_ERR_UNSUPPORTED
+
+
+def test_share_output_validated_on_the_host():
+    import ctypes
+    lib = dt.load()
+    base = 1 << 20
+    assert lib.dt_share_output(0, 1024, 64, None, None, None, None, None) == dt.DT_OK          # nothing to copy
+    assert lib.dt_share_output(-1, 1024, 64, base, base, base, base, None) == dt.DT_ERR_INVALID
+    assert lib.dt_share_output(2, 1024, 64, None, base, base, base, None) == dt.DT_ERR_INVALID
+    # partially overlapping ranges are refused; identical ones are a no-op
+    assert lib.dt_share_output(2, 1024, 64, base, base * 8, base + 4096, base * 16, None) == dt.DT_ERR_INVALID
+    assert lib.dt_share_output(2, 1024, 64, base, base * 8, base, base * 8, None) == dt.DT_OK

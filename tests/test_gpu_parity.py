@@ -431,3 +431,55 @@ def test_importance_weights_and_plan_match_oracle(H, S, D, P, g):
         run_partition_schedule(H, S, D, P, [(step, dt.DT_MODE_IMPORTANCE, 2, None)], lambda: next(it),
                                check_untouched=True, sess=sess, cache=cache)
         np.testing.assert_array_equal(sess.last_plan, want)
+
+
+# ------------------------------------------------------- attention sharing
+
+@pytest.mark.parametrize("g", [0, 2])
+def test_cfg_shared_step(g):
+    """Sharing across CFG branches: heads [0, H/2) (conditional) are computed
+    and match the oracle on their own inputs; heads [H/2, H) receive the same
+    bytes, their inputs are ignored and their cache slots stay untouched."""
+    Hb, S, D, P = 2, 1024, 64, 4
+    r = 1
+    cond = wl.InputStream(Hb, S, D, 0.05, seed=90)
+    other = wl.InputStream(Hb, S, D, 0.5, seed=91)
+    sess = Session(2 * Hb, S, D, P, reuse_per_row=r, group=g)
+    cache = orc.StateCache()
+    for step in (1, 2):
+        qc, kc, vc = cond.next_step()
+        qu, ku, vu = other.next_step()
+        sess.set_inputs(*(np.concatenate([a, b]) for a, b in ((qc, qu), (kc, ku), (vc, vu))))
+        sess.counters.zero_()
+        counts = sess.step_cfg_shared(step)
+        sess.check()
+        O_ref, L_ref, _ = orc.partition_step(qc, kc, vc, sess.last_plan, S, P, cache, group=g)
+        check_out(to_np(sess.O[:Hb]), O_ref, f"cond O step {step}")
+        check_lse(to_np(sess.L[:Hb]), L_ref, f"cond LSE step {step}")
+        assert torch.equal(sess.O[Hb:].view(torch.int16), sess.O[:Hb].view(torch.int16))
+        assert torch.equal(sess.L[Hb:], sess.L[:Hb])
+        assert torch.all(sess.cache_O[:, Hb:] == 0) and torch.all(torch.isneginf(sess.cache_L[:, Hb:]))
+        c = sess.counters.cpu().numpy()
+        assert int(c[0]) == counts["computed_blocks"]
+        assert counts["computed_blocks"] + counts["skipped_blocks"] == \
+            2 * Hb * sum(orc.n_kv_tiles(a, b) for a, b in orc.partitions(S, P)) * len(orc.query_tiles(S, P))
+
+
+def test_share_previous_output():
+    """Sharing across timesteps: nothing is launched; O and L keep the
+    previous step's bytes and every block counts as skipped."""
+    w = wl.WORKLOADS[0]
+    sess = Session(w.H, w.S, w.D, w.P, reuse_per_row=2)
+    s = wl.stream_for(w)
+    for step in (1, 2):
+        sess.set_inputs(*s.next_step())
+        sess.step(step)
+    sess.check()
+    o, l, st = sess.O.clone(), sess.L.clone(), sess.stamps.copy()
+    sess.set_inputs(*s.next_step())
+    counts = sess.share_previous_output()
+    sess.check()
+    assert torch.equal(sess.O.view(torch.int16), o.view(torch.int16)) and torch.equal(sess.L, l)
+    assert np.array_equal(sess.stamps, st)
+    assert counts["computed_blocks"] == 0 and counts["computed_flops"] == 0
+    assert counts["skipped_blocks"] == w.H * 8 * 8
