@@ -133,6 +133,18 @@ DT_API const char* dt_status_string(int status);
  * partitioning of the sequence).  Host only.  Errors: DT_ERR_INVALID. */
 DT_API int dt_plan_geometry(const dt_plan_params* p, int32_t* nqt, int32_t* nseg);
 
+/* Key tiles of key set k of query tile qt, as the fused kernel visits them
+ * (before its rotation of the visiting order): for tile i, rows
+ * [row0[i], min(row0[i] + 128, rowend[i])) of K and V.  Tiles are
+ * partition-local; a grouped set lists its partitions' tiles in increasing
+ * partition order, skipping the query's own partition.  Window mode lists
+ * the tiles of its two key sets (edge tiles then carry a band mask not
+ * shown here).  Fills at most cap entries of row0 / rowend (host arrays,
+ * NULL if cap = 0) and returns the number of tiles (>= 0), or DT_ERR_INVALID.
+ * Host only. */
+DT_API int dt_key_set_tiles(const dt_plan_params* p, int32_t qt, int32_t k, int32_t* row0, int32_t* rowend,
+                     int32_t cap);
+
 /* Build the compute/reuse plan of one step on the host ("DiTango", selective
  * compute and reuse, Fig. 6; anchor steps).  explicit_plan ([nqt][nseg],
  * values DT_PLAN_*) is read only in DT_MODE_EXPLICIT.  Window mode: key set 0

@@ -25,7 +25,7 @@ __all__ = [
     "DT_ERR_TIMEOUT", "DT_MODE_ALL_COMPUTE", "DT_MODE_PROXIMITY", "DT_MODE_ALL_REUSE",
     "DT_MODE_EXPLICIT", "DT_MODE_WINDOW", "DT_PLAN_REUSE", "DT_PLAN_COMPUTE", "DT_WR_MAKE",
     "DT_WR_APPLY", "DT_TILE", "DT_STATE_F32", "DT_STATE_BF16", "DT_MODE_IMPORTANCE",
-    "dt_plan_build_importance", "dt_state_importance", "dt_share_output",
+    "dt_plan_build_importance", "dt_state_importance", "dt_share_output", "dt_key_set_tiles",
 ]
 
 DT_OK, DT_ERR_INVALID, DT_ERR_UNSUPPORTED, DT_ERR_CACHE_EMPTY, DT_ERR_CUDA, DT_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
@@ -86,6 +86,7 @@ def load() -> ctypes.CDLL:
             "dt_plan_build_importance": ([pp, vp, ctypes.POINTER(Plan)], ctypes.c_int),
             "dt_state_importance": ([pp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_share_output": ([i32, i32, i32, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_key_set_tiles": ([pp, i32, i32, vp, vp, i32], ctypes.c_int),
             "dt_set_wait_limit_ns": ([i64], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -172,6 +173,18 @@ def dt_plan_build_importance(p: PlanParams, weights: Optional[np.ndarray], stamp
 def dt_state_importance(p: PlanParams, cache_L, L, d_weights, d_status=None, stream=None) -> None:
     _check(load().dt_state_importance(ctypes.byref(p), _ptr(cache_L), _ptr(L), _ptr(d_weights), _ptr(d_status),
                                       _stream(stream)), "dt_state_importance")
+
+
+def dt_key_set_tiles(p: PlanParams, qt: int, k: int):
+    """Key tiles of key set k of query tile qt: list of (row0, rowend) with
+    the tile's rows [row0, min(row0 + 128, rowend))."""
+    n = load().dt_key_set_tiles(ctypes.byref(p), qt, k, None, None, 0)
+    if n < 0:
+        raise DtError(n, "dt_key_set_tiles")
+    r0 = np.zeros(max(n, 1), np.int32)
+    re = np.zeros(max(n, 1), np.int32)
+    load().dt_key_set_tiles(ctypes.byref(p), qt, k, r0.ctypes.data, re.ctypes.data, n)
+    return list(zip(r0[:n].tolist(), re[:n].tolist()))
 
 
 def dt_share_output(n_heads: int, S: int, D: int, src_O, src_L, dst_O, dst_L, stream=None) -> None:

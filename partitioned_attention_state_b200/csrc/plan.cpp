@@ -99,6 +99,21 @@ extern "C" const char* dt_status_string(int s) {
   }
 }
 
+extern "C" int dt_key_set_tiles(const dt_plan_params* p, int32_t qt, int32_t k, int32_t* row0, int32_t* rowend,
+                                int32_t cap) {
+  if (!params_ok(p) || cap < 0 || (cap > 0 && (!row0 || !rowend))) return DT_ERR_INVALID;
+  dt::Geom g = geom_of(p);
+  if (qt < 0 || qt >= g.nqt || k < 0 || k >= g.P) return DT_ERR_INVALID;
+  const dt::KeySet ks = dt::key_set(g, qt, k);
+  const int nt = ks.ntiles();
+  for (int i = 0; i < nt && i < cap; ++i) {
+    const int t = ks.tile(i);
+    row0[i] = ks.row0(t);
+    rowend[i] = ks.rowend(t);
+  }
+  return nt;
+}
+
 extern "C" int dt_plan_geometry(const dt_plan_params* p, int32_t* nqt, int32_t* nseg) {
   if (!params_ok(p) || !nqt || !nseg) return DT_ERR_INVALID;
   dt::Geom g = geom_of(p);

@@ -325,3 +325,64 @@ def test_share_output_validated_on_the_host():
     # partially overlapping ranges are refused; identical ones are a no-op
     assert lib.dt_share_output(2, 1024, 64, base, base * 8, base + 4096, base * 16, None) == dt.DT_ERR_INVALID
     assert lib.dt_share_output(2, 1024, 64, base, base * 8, base, base * 8, None) == dt.DT_OK
+
+
+def expected_partition_tiles(S, P, ks):
+    """Partition-local 128-row tiles of the partitions of a key set, in order."""
+    parts = orc.partitions(S, P)
+    out = []
+    for p in ks:
+        a, b = parts[p]
+        out += [(r, min(r + 128, b)) for r in range(a, b, 128)]
+    return out
+
+
+@pytest.mark.parametrize("S,P", [(1024, 4), (1000, 3), (5, 4), (2600, 64), (1800, 12), (32760, 16), (4097, 7),
+                                 (300, 5), (129, 2), (100, 60), (640, 8)])
+def test_key_set_tiles_match_oracle_key_sets(S, P):
+    """The tiles the kernel visits for each (query tile, key set), from the
+    same geometry code, cover exactly the oracle's key set: per partition,
+    grouped (every group size), ungrouped."""
+    for g in sorted({0, 1, 2, 3, 5, P}):
+        p = dt.params(1, S, 64, P, dt.DT_MODE_ALL_COMPUTE, 0, 0, 1, g)
+        nqt, nseg = dt.dt_plan_geometry(p)
+        tiles = orc.query_tiles(S, P)
+        for qt in range(0, nqt, max(1, nqt // 17)):
+            sets = orc.key_sets_of_tile(tiles[qt][0], P, g)
+            assert len(sets) == nseg
+            for k in range(nseg):
+                got = [(a, min(a + 128, e)) for a, e in dt.dt_key_set_tiles(p, qt, k)]
+                assert got == expected_partition_tiles(S, P, sets[k]), (S, P, g, qt, k)
+
+
+@pytest.mark.parametrize("S,W", [(16384, 1024), (1000, 100), (300, 64), (129, 1), (200, 400), (5000, 129)])
+def test_window_key_set_tiles_by_brute_force(S, W):
+    """Window mode: set 0 holds every key tile with a (query, key) pair inside
+    the band, set 1 every key tile with a pair outside it (brute force over
+    all pairs of the query tile)."""
+    p = dt.params(1, S, 64, 1, dt.DT_MODE_WINDOW, 0, W, 1)
+    nqt, _ = dt.dt_plan_geometry(p)
+    keys = np.arange(S)
+    for qt in range(0, nqt, max(1, nqt // 13)):
+        rows = np.arange(qt * 128, min(qt * 128 + 128, S))
+        inside = orc.window_in(rows, keys, W)
+        want0, want1 = [], []
+        for t in range(0, S, 128):
+            blk = inside[:, t:t + 128]
+            if blk.any():
+                want0.append((t, min(t + 128, S)))
+            if not blk.all():
+                want1.append((t, min(t + 128, S)))
+        got0 = sorted((a, min(a + 128, e)) for a, e in dt.dt_key_set_tiles(p, qt, 0))
+        got1 = sorted((a, min(a + 128, e)) for a, e in dt.dt_key_set_tiles(p, qt, 1))
+        assert got0 == want0 and got1 == want1, (S, W, qt)
+
+
+def test_key_set_tiles_validated():
+    import ctypes
+    lib = dt.load()
+    p = dt.params(1, 1024, 64, 4, dt.DT_MODE_ALL_COMPUTE, 0, 0, 1)
+    for qt, k in ((-1, 0), (8, 0), (0, 4), (0, -1)):
+        assert lib.dt_key_set_tiles(ctypes.byref(p), qt, k, None, None, 0) == dt.DT_ERR_INVALID
+    assert lib.dt_key_set_tiles(ctypes.byref(p), 0, 0, None, None, 1) == dt.DT_ERR_INVALID
+    assert lib.dt_key_set_tiles(ctypes.byref(p), 0, 0, None, None, 0) == 2
