@@ -5,8 +5,12 @@ residual, outputs, counters, status word) and the host stamps, and runs one
 denoising step as: host plan build (``dt_plan_build``) -> plan upload ->
 one fused launch (``dt_attn_partial_fused``), or, from host buffers, as
 head-group launches (``dt_attn_partial_fused_heads``) pipelined with their
-copies.  torch provides the memory and the streams; every computation
-happens in libdt.
+copies.  The key sets are partitions or groups of partitions (``group``),
+the cached OUT fp32 or bf16 (``state_dtype``); plans follow the proximity
+rule, an explicit plan, or measured importance (``measure_importance``);
+cached group states can be regrouped (``compose_groups``) and outputs shared
+across CFG branches or timesteps.  torch provides the memory and the
+streams; every computation happens in libdt.
 """
 
 from __future__ import annotations
@@ -28,6 +32,9 @@ def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
 
 
 class Session:
+    """Buffers, host stamps and plan state of one stream of denoising steps
+    of one attention layer."""
+
     def __init__(self, H: int, S: int, D: int, P: int = 1, mode: int = DT_MODE_PROXIMITY, reuse_per_row: int = 0,
                  window: int = 0, device: str = "cuda", cache: bool = True, group: int = 0,
                  state_dtype: int = 0):
