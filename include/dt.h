@@ -175,7 +175,9 @@ DT_API int dt_plan_build_importance(const dt_plan_params* p, const float* weight
  * or a window-mode set): COMPUTE runs the partial attention (tensor cores) and
  * writes the fresh state (OUT, LSE) to its cache slot; REUSE reads the cached
  * state.  All states of the row are composed into O (bf16) and L.
- *   d_plan      device copy of dt_plan.plan, [nqt][nseg] uint8
+ *   d_plan      device copy of dt_plan.plan, [nqt][nseg] uint8; every entry
+ *               must be DT_PLAN_REUSE (0) or DT_PLAN_COMPUTE (1) (the kernel
+ *               reads bit 0 of each byte; dt_plan_build writes only 0 and 1)
  *   Q, K, V     bf16 [H][S][D] (read)
  *   cache_O/L   fp32 [nseg][H][S][D] / [nseg][H][S] state slots, slot (k, h,
  *               row) for key set k (REUSE slots read, COMPUTE slots written;
@@ -280,6 +282,39 @@ DT_API int dt_window_residual(int32_t op, int32_t H, int32_t S, int32_t D,
  * null or partially overlapping buffers), DT_ERR_CUDA. */
 DT_API int dt_share_output(int32_t n_heads, int32_t S, int32_t D, const void* src_O, const float* src_L,
                     void* dst_O, float* dst_L, void* stream);
+
+/* Attention sharing across CFG branches as one step ("DiTFastAttn",
+ * attention sharing across CFG: the unconditional branch takes the
+ * conditional branch's attention output).  The p->H heads (H even) hold the
+ * conditional branch in heads [0, H/2) and the unconditional one in
+ * [H/2, H).  Runs the fused step (arguments as dt_attn_partial_fused, with
+ * the plan dt_plan_build made for all H heads) on the conditional heads,
+ * copies their O and L to the unconditional heads, and copies the states
+ * they computed (cache slots of the COMPUTE entries; in window mode R rows
+ * where the complement was computed) to the same slots of the unconditional
+ * heads: the shared attention is the conditional branch's, so the stamps
+ * dt_plan_build wrote stay true for every head, and a later step that
+ * computes both branches reuses those states.  Unconditional inputs are not
+ * read.  The counters accumulate the conditional heads' launch.  Errors:
+ * those of dt_attn_partial_fused, DT_ERR_INVALID for odd H. */
+DT_API int dt_attn_cfg_shared(const dt_plan_params* p, const uint8_t* d_plan,
+                       const void* Q, const void* K, const void* V,
+                       float* cache_O, float* cache_L, float* R, void* O, float* L,
+                       int64_t* d_counters, int32_t* d_status, void* stream);
+
+#define DT_SHARE_CFG      0   /* the conditional half computes, the unconditional half shares */
+#define DT_SHARE_TIMESTEP 1   /* the step takes the previous step's output: nothing computed */
+
+/* Counts of a step that shares attention ("DiTFastAttn", attention sharing
+ * across CFG branches and across timesteps).  DT_SHARE_CFG: on entry io
+ * holds the counts dt_plan_build returned for the step's plan over all p->H
+ * heads (H even); on return, the counts of the step as dt_attn_cfg_shared
+ * runs it (the unconditional half's blocks skipped, its FLOPs not spent).
+ * DT_SHARE_TIMESTEP: io's counts become zero computed blocks and FLOPs and
+ * every block of every head skipped (counts on entry ignored).  io->plan and
+ * io->stamps are neither read nor written.  Host only.  Errors:
+ * DT_ERR_INVALID (bad params, unknown kind, odd H for DT_SHARE_CFG). */
+DT_API int dt_plan_share_counts(const dt_plan_params* p, int32_t kind, dt_plan* io);
 
 /* Limit, in nanoseconds, of every bounded wait inside the fused kernel
  * (default 2e9).  A wait that runs out writes DT_ERR_TIMEOUT to *d_status and

@@ -26,6 +26,7 @@ __all__ = [
     "DT_MODE_EXPLICIT", "DT_MODE_WINDOW", "DT_PLAN_REUSE", "DT_PLAN_COMPUTE", "DT_WR_MAKE",
     "DT_WR_APPLY", "DT_TILE", "DT_STATE_F32", "DT_STATE_BF16", "DT_MODE_IMPORTANCE",
     "dt_plan_build_importance", "dt_state_importance", "dt_share_output", "dt_key_set_tiles",
+    "dt_attn_cfg_shared", "dt_plan_share_counts", "DT_SHARE_CFG", "DT_SHARE_TIMESTEP",
 ]
 
 DT_OK, DT_ERR_INVALID, DT_ERR_UNSUPPORTED, DT_ERR_CACHE_EMPTY, DT_ERR_CUDA, DT_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
@@ -34,6 +35,7 @@ DT_STATE_F32, DT_STATE_BF16 = 0, 1
 DT_MODE_ALL_COMPUTE, DT_MODE_PROXIMITY, DT_MODE_ALL_REUSE, DT_MODE_EXPLICIT, DT_MODE_WINDOW = 0, 1, 2, 3, 4
 DT_PLAN_REUSE, DT_PLAN_COMPUTE = 0, 1
 DT_WR_MAKE, DT_WR_APPLY = 0, 1
+DT_SHARE_CFG, DT_SHARE_TIMESTEP = 0, 1
 DT_TILE = 128
 
 
@@ -86,6 +88,8 @@ def load() -> ctypes.CDLL:
             "dt_plan_build_importance": ([pp, vp, ctypes.POINTER(Plan)], ctypes.c_int),
             "dt_state_importance": ([pp, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_share_output": ([i32, i32, i32, vp, vp, vp, vp, vp], ctypes.c_int),
+            "dt_attn_cfg_shared": ([pp] + [vp] * 12, ctypes.c_int),
+            "dt_plan_share_counts": ([pp, i32, ctypes.POINTER(Plan)], ctypes.c_int),
             "dt_key_set_tiles": ([pp, i32, i32, vp, vp, i32], ctypes.c_int),
             "dt_set_wait_limit_ns": ([i64], ctypes.c_int),
         }
@@ -190,6 +194,27 @@ def dt_key_set_tiles(p: PlanParams, qt: int, k: int):
 def dt_share_output(n_heads: int, S: int, D: int, src_O, src_L, dst_O, dst_L, stream=None) -> None:
     _check(load().dt_share_output(n_heads, S, D, _ptr(src_O), _ptr(src_L), _ptr(dst_O), _ptr(dst_L),
                                   _stream(stream)), "dt_share_output")
+
+
+def dt_attn_cfg_shared(p: PlanParams, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,
+                       stream=None) -> None:
+    _check(load().dt_attn_cfg_shared(ctypes.byref(p), _ptr(d_plan), _ptr(Q), _ptr(K), _ptr(V), _ptr(cache_O),
+                                     _ptr(cache_L), _ptr(R), _ptr(O), _ptr(L), _ptr(d_counters), _ptr(d_status),
+                                     _stream(stream)), "dt_attn_cfg_shared")
+
+
+def dt_plan_share_counts(p: PlanParams, kind: int, counts: Optional[dict] = None) -> dict:
+    """Counts of a step under attention sharing (DT_SHARE_CFG: from the
+    counts of the step's plan over all heads; DT_SHARE_TIMESTEP: nothing
+    computed)."""
+    io = Plan()
+    if counts is not None:
+        io.computed_blocks = counts["computed_blocks"]
+        io.skipped_blocks = counts["skipped_blocks"]
+        io.computed_flops = counts["computed_flops"]
+    _check(load().dt_plan_share_counts(ctypes.byref(p), kind, ctypes.byref(io)), "dt_plan_share_counts")
+    return {"computed_blocks": io.computed_blocks, "skipped_blocks": io.skipped_blocks,
+            "computed_flops": io.computed_flops}
 
 
 def dt_attn_partial_fused(p: PlanParams, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,

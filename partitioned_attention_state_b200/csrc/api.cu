@@ -252,6 +252,27 @@ extern "C" int dt_share_output(int32_t n_heads, int32_t S, int32_t D, const void
   return DT_OK;
 }
 
+extern "C" int dt_attn_cfg_shared(const dt_plan_params* p, const uint8_t* d_plan, const void* Q, const void* K,
+                                  const void* V, float* cache_O, float* cache_L, float* R, void* O, float* L,
+                                  int64_t* d_counters, int32_t* d_status, void* stream) {
+  if (!p || p->H % 2 != 0) return DT_ERR_INVALID;
+  const int hb = p->H / 2;
+  if (int e = dt_attn_partial_fused_heads(p, 0, hb, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,
+                                          stream))
+    return e;
+  if (hb == 0 || p->S == 0) return DT_OK;
+  const size_t half = (size_t)hb * p->S;
+  if (int e = dt_share_output(hb, p->S, p->D, O, L, static_cast<uint16_t*>(O) + half * p->D, L + half, stream))
+    return e;
+  const bool win = p->mode == DT_MODE_WINDOW;
+  const dt::Geom G = dt::make_geom(p->H, p->S, p->D, win ? 1 : p->P, win ? p->window : 0, win ? 0 : p->group);
+  int sms = 0;
+  if (int e = sm_count(&sms)) return e;
+  const int elem = win ? 4 : (p->state_dtype == DT_STATE_BF16 ? 2 : 4);
+  return dt::launch_share_states(G, d_plan, hb, elem, cache_O, cache_L, R, sms,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" int dt_window_residual(int32_t op, int32_t H, int32_t S, int32_t D, const float* O_full,
                                   const float* O_win, float* R, void* O, int32_t* d_status, void* stream) {
   if (op != DT_WR_MAKE && op != DT_WR_APPLY) return DT_ERR_INVALID;

@@ -63,6 +63,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/dt.h"
 #include "attn_fused.h"
 #include "exp2_poly.h"
@@ -84,6 +86,7 @@ constexpr int kLaunchRegs = 128;
 constexpr int kRegsSoftmax = 128, kRegsEpilogue = 192, kRegsOther = 64;
 static_assert(128 * (2 * kRegsSoftmax + kRegsEpilogue + kRegsOther) <= kThreads * kLaunchRegs, "register split");
 constexpr uint64_t kDrainLimitNs = 1000000000ull;   // drains use a fixed limit
+constexpr int kMaxDevices = 64;
 __device__ __forceinline__ float neg_inf() { return -__int_as_float(0x7f800000); }
 #define kNegInf (neg_inf())
 constexpr float kLog2e = 1.4426950408889634f;
@@ -167,13 +170,14 @@ __device__ __forceinline__ uint32_t mask4(uint32_t w) {     // 4 plan bytes (0/1
 template <bool WIN>
 __device__ __forceinline__ uint64_t plan_mask(const uint8_t* prow, int P) {
   uint64_t m = 0;
+  // every loader reads bit 0 of a plan byte (DT_PLAN_COMPUTE = 1, DT_PLAN_REUSE = 0)
   if (WIN) {                                // two key sets
-    m = (uint64_t)(prow[0] == DT_PLAN_COMPUTE) | ((uint64_t)(prow[1] == DT_PLAN_COMPUTE) << 1);
+    m = (uint64_t)(prow[0] & 1u) | ((uint64_t)(prow[1] & 1u) << 1);
   } else if ((P & 3) == 0) {                // rows start 4-byte aligned
 #pragma unroll 4
     for (int s = 0; s < P; s += 4) m |= (uint64_t)mask4(*reinterpret_cast<const uint32_t*>(prow + s)) << s;
   } else {
-    for (int s = 0; s < P; ++s) m |= (uint64_t)(prow[s] == DT_PLAN_COMPUTE) << s;
+    for (int s = 0; s < P; ++s) m |= (uint64_t)(prow[s] & 1u) << s;
   }
   return m;
 }
@@ -757,6 +761,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         n_comp += counted_blocks<KM>(G, qt, seg);
         ++n_fresh;
         if (nt == 0) {             // empty key set: the identity state
+          if (WIN && valid && seg == 1) {
+            // empty complement (the band covers every key of the row's
+            // tile): full attention equals window attention, so R = 0
+            float4* dst = reinterpret_cast<float4*>(p.R + ((size_t)h * G.S + qrow) * D);
+            for (int d = 0; d < D / 4; ++d) __stcs(dst + d, make_float4(0.f, 0.f, 0.f, 0.f));
+          }
           if (!WIN && valid) {
             if (CBF) {
               uint2* dst = reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.cache_O) + slot * D);
@@ -874,12 +884,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 template <int DP, int MODE>
 int launch_dp(const AttnParams& kp, int grid, cudaStream_t stream) {
   using C = Cfg<DP>;
-  static bool attr_set = false;   // per-process; the attribute is per device function
-  if (!attr_set) {
+  // The shared-memory attribute belongs to the function on each device: set
+  // it once per device (a repeated set from racing threads is harmless).
+  static std::atomic<bool> attr_set[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DT_ERR_CUDA;
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (!cached || !attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(attn_partial_fused_kernel<DP, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmem) != cudaSuccess)
       return DT_ERR_CUDA;
-    attr_set = true;
+    if (cached) attr_set[dev].store(true, std::memory_order_release);
   }
   attn_partial_fused_kernel<DP, MODE><<<grid, kThreads, C::kSmem, stream>>>(kp);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;

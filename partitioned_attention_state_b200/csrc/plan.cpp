@@ -199,6 +199,29 @@ extern "C" int dt_plan_build_importance(const dt_plan_params* p, const float* we
   return finish_plan(p, g, out);
 }
 
+
+extern "C" int dt_plan_share_counts(const dt_plan_params* p, int32_t kind, dt_plan* io) {
+  if (!params_ok(p) || !io) return DT_ERR_INVALID;
+  if (kind == DT_SHARE_CFG) {
+    // the plan's counts are H x (per-head counts), so halving is exact
+    if (p->H % 2 != 0) return DT_ERR_INVALID;
+    const int64_t total = io->computed_blocks + io->skipped_blocks;
+    io->computed_blocks /= 2;
+    io->skipped_blocks = total - io->computed_blocks;
+    io->computed_flops /= 2;
+    return DT_OK;
+  }
+  if (kind != DT_SHARE_TIMESTEP) return DT_ERR_INVALID;
+  const dt::Geom g = geom_of(p);
+  int64_t total = 0;
+  for (int qt = 0; qt < g.nqt; ++qt)
+    for (int k = 0; k < g.P; ++k) total += (int64_t)p->H * dt::counted_blocks(g, qt, k);
+  io->computed_blocks = 0;
+  io->skipped_blocks = total;
+  io->computed_flops = 0;
+  return DT_OK;
+}
+
 namespace {
 
 // Shared tail of the plan builders: refuse REUSE of never-written slots,

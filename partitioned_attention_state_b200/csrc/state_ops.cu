@@ -195,6 +195,50 @@ __global__ void __launch_bounds__(kBlock) state_importance_kernel(Geom G, const 
   }
 }
 
+// "DiTFastAttn", attention sharing across CFG branches: the unconditional
+// branch takes the conditional branch's attention, so the states the
+// conditional heads computed this step also become the unconditional heads'
+// cached states.  For every (query tile, key set) the plan marks COMPUTE,
+// the slot rows of head h < hb are copied to head h + hb (cache_O as fp32 or
+// bf16, cache_L fp32); in window mode a computed complement copies the rows
+// of R instead.  One thread per 16-byte vector.
+__global__ void __launch_bounds__(kBlock) share_states_kernel(Geom G, const uint8_t* __restrict__ plan, int hb,
+                                                              int elem_bytes, uint8_t* __restrict__ cO,
+                                                              float* __restrict__ cL, float* __restrict__ R) {
+  const bool win = G.window > 0;
+  const int vec = 16 / elem_bytes;                       // elements per 16-byte vector
+  const int dv = G.D / vec;
+  const int nk = win ? 1 : G.P;
+  const int64_t rows = (int64_t)nk * hb * G.S;
+  const int64_t total = rows * dv;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / dv;                          // ((k * hb + h) * S + s)
+    const int c = (int)(i - row * dv);
+    const int s = (int)(row % G.S);
+    const int h = (int)((row / G.S) % hb);
+    const int k = (int)(row / ((int64_t)hb * G.S));
+    int qt;
+    if (win) {
+      qt = s / kTile;
+    } else {
+      const int part = s / G.c;
+      qt = part * G.tpp + (s - part_begin(G, part)) / kTile;
+    }
+    const int seg = win ? 1 : k;
+    if ((plan[(size_t)qt * G.P + seg] & 1u) == 0) continue;
+    if (win) {
+      const float4* src = reinterpret_cast<const float4*>(R + ((int64_t)h * G.S + s) * G.D);
+      float4* dst = reinterpret_cast<float4*>(R + ((int64_t)(h + hb) * G.S + s) * G.D);
+      dst[c] = src[c];
+    } else {
+      const int64_t from = ((int64_t)k * G.H + h) * G.S + s, to = ((int64_t)k * G.H + h + hb) * G.S + s;
+      reinterpret_cast<uint4*>(cO + to * G.D * elem_bytes)[c] =
+          reinterpret_cast<const uint4*>(cO + from * G.D * elem_bytes)[c];
+      if (c == 0) cL[to] = cL[from];
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kBlock) fill_zero_kernel(float* __restrict__ x, int64_t n) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
     x[i] = 0.f;
@@ -239,6 +283,16 @@ int launch_group_compose(int m, int factor, int H, int S, int D, float* cO, floa
 int launch_state_importance(const Geom& G, const float* cL, const float* L, float* w, cudaStream_t st) {
   const int64_t blocks = (int64_t)G.nqt * G.P;
   state_importance_kernel<<<(unsigned)blocks, kBlock, 0, st>>>(G, cL, L, w);
+  return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+}
+
+int launch_share_states(const Geom& G, const uint8_t* plan, int hb, int elem_bytes, void* cO, float* cL, float* R,
+                        int sms, cudaStream_t st) {
+  const int nk = G.window > 0 ? 1 : G.P;
+  const int64_t work = (int64_t)nk * hb * G.S * (G.D * elem_bytes / 16);
+  if (work == 0) return DT_OK;
+  share_states_kernel<<<grid_for(work, sms), kBlock, 0, st>>>(G, plan, hb, elem_bytes,
+                                                              reinterpret_cast<uint8_t*>(cO), cL, R);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
 }
 

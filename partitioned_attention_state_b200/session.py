@@ -20,9 +20,10 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (DT_MODE_IMPORTANCE, DT_MODE_PROXIMITY, DT_MODE_WINDOW, dt_attn_partial_fused,
-               dt_attn_partial_fused_heads, dt_group_compose, dt_plan_build, dt_plan_build_importance, dt_plan_geometry,
-               dt_share_output, dt_state_importance, DtError, params)
+from . import (DT_MODE_IMPORTANCE, DT_MODE_PROXIMITY, DT_MODE_WINDOW, DT_SHARE_CFG, DT_SHARE_TIMESTEP,
+               dt_attn_cfg_shared, dt_attn_partial_fused, dt_attn_partial_fused_heads, dt_group_compose,
+               dt_plan_build, dt_plan_build_importance, dt_plan_geometry, dt_plan_share_counts, dt_state_importance,
+               DtError, params)
 
 
 def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
@@ -81,6 +82,7 @@ class Session:
                         for _ in range(2)]
         self._uploaded = [None, None]
         self._turn = 0
+        self._plan_read = None       # event after the last launch that read d_plan
 
     def compose_groups(self, factor: int = 2, shrink: bool = False) -> None:
         """Dynamic Group State Compose: regroup the cached group states into
@@ -141,13 +143,17 @@ class Session:
              stream=None) -> dict:
         """Host plan build, asynchronous plan upload, one fused launch."""
         p, plan, counts = self.plan(step, mode, explicit)
-        self._upload_plan(plan, torch.cuda.current_stream(self.device) if stream is None else stream)
-        self.launch(p, stream)
+        st = torch.cuda.current_stream(self.device) if stream is None else stream
+        self._upload_plan(plan, st)
+        self.launch(p, st)
+        self._mark_plan_read(st)
         self.last_counts, self.last_plan = counts, plan
         return counts
 
     def _upload_plan(self, plan: np.ndarray, st) -> None:
-        """Asynchronous copy of a host plan into d_plan, ordered on stream `st`."""
+        """Asynchronous copy of a host plan into d_plan, ordered on stream `st`
+        after the previous launch that read d_plan (which may have been
+        issued on another stream)."""
         if self.nqt == 0:
             return
         i = self._turn
@@ -156,11 +162,19 @@ class Session:
             self._uploaded[i].synchronize()      # that buffer's previous upload is done
         buf = self._pinned[i]
         buf[: self.nqt].numpy()[...] = plan
+        if self._plan_read is not None:
+            st.wait_event(self._plan_read)
         with torch.cuda.stream(st):
             self.d_plan[: self.nqt].copy_(buf[: self.nqt], non_blocking=True)
             ev = torch.cuda.Event()
             ev.record(st)
         self._uploaded[i] = ev
+
+    def _mark_plan_read(self, st) -> None:
+        """Record that the launches issued so far on `st` read d_plan."""
+        ev = torch.cuda.Event()
+        ev.record(st)
+        self._plan_read = ev
 
     def step_host(self, step: int, q, k, v, o, lse, groups: Optional[int] = None, mode: Optional[int] = None,
                   explicit: Optional[np.ndarray] = None) -> dict:
@@ -214,6 +228,7 @@ class Session:
             with torch.cuda.stream(down):
                 o[h0:h1].copy_(dev_view(self.O, o)[h0:h1], non_blocking=True)
                 lse[h0:h1].copy_(self.L[h0:h1], non_blocking=True)
+        self._mark_plan_read(comp)
         for st in self._host_streams:
             cur.wait_stream(st)
         self.last_counts, self.last_plan = counts, plan
@@ -221,26 +236,23 @@ class Session:
 
     def step_cfg_shared(self, step: int, mode: Optional[int] = None, explicit: Optional[np.ndarray] = None,
                         stream=None) -> dict:
-        """Attention sharing across CFG branches: the session's H heads are the
-        conditional half [0, H/2) and the unconditional half [H/2, H) of one
-        layer.  Only the conditional half is computed (plan, cache slots and
-        stamps as in step()); its O and L are then copied to the unconditional
-        half, whose inputs are not read and whose cache slots stay untouched.
-        Returns the counts of the whole batch, the unconditional half's blocks
-        counted as skipped."""
+        """Attention sharing across CFG branches (dt_attn_cfg_shared): the
+        session's H heads are the conditional half [0, H/2) and the
+        unconditional half [H/2, H) of one layer.  The conditional half is
+        computed with the step's plan; its O and L, and the states it
+        computed, are copied to the unconditional half (whose inputs are not
+        read), so the stamps hold for every head and later steps may compute
+        both halves.  Returns the counts of the whole batch, the
+        unconditional half's blocks counted as skipped (dt_plan_share_counts)."""
         if self.H % 2:
             raise ValueError("CFG sharing needs an even number of heads (two branches)")
-        hb = self.H // 2
         p, plan, counts = self.plan(step, mode, explicit)
         st = torch.cuda.current_stream(self.device) if stream is None else stream
         self._upload_plan(plan, st)
-        dt_attn_partial_fused_heads(p, 0, hb, self.d_plan, self.Q, self.K, self.V, self.cache_O, self.cache_L,
-                                    self.R, self.O, self.L, self.counters, self.status, st)
-        dt_share_output(hb, self.S, self.D, self.O[:hb], self.L[:hb], self.O[hb:], self.L[hb:], st)
-        total = counts["computed_blocks"] + counts["skipped_blocks"]
-        out = {"computed_blocks": counts["computed_blocks"] // 2,
-               "skipped_blocks": total - counts["computed_blocks"] // 2,
-               "computed_flops": counts["computed_flops"] // 2}
+        dt_attn_cfg_shared(p, self.d_plan, self.Q, self.K, self.V, self.cache_O, self.cache_L, self.R, self.O,
+                           self.L, self.counters, self.status, st)
+        self._mark_plan_read(st)
+        out = dt_plan_share_counts(p, DT_SHARE_CFG, counts)
         self.last_counts, self.last_plan = out, plan
         return out
 
@@ -248,14 +260,11 @@ class Session:
         """Attention sharing across timesteps: this step takes the previous
         step's attention output, which O and L already hold.  Nothing is
         launched; plan, cache and stamps are untouched.  Returns the counts
-        (every block skipped, no FLOPs)."""
+        (every block skipped, no FLOPs; dt_plan_share_counts)."""
         win = self.mode == DT_MODE_WINDOW
-        p = params(self.H, self.S, self.D, 1 if win else self.P, 0, 0, self.window, 1, 0 if win else self.group)
-        if win:
-            p.mode = DT_MODE_WINDOW
-        _, full = dt_plan_build(p, None)
-        out = {"computed_blocks": 0, "skipped_blocks": full["computed_blocks"] + full["skipped_blocks"],
-               "computed_flops": 0}
+        p = params(self.H, self.S, self.D, 1 if win else self.P, DT_MODE_WINDOW if win else 0, 0, self.window, 1,
+                   0 if win else self.group)
+        out = dt_plan_share_counts(p, DT_SHARE_TIMESTEP)
         self.last_counts = out
         return out
 

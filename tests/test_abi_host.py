@@ -386,3 +386,48 @@ def test_key_set_tiles_validated():
         assert lib.dt_key_set_tiles(ctypes.byref(p), qt, k, None, None, 0) == dt.DT_ERR_INVALID
     assert lib.dt_key_set_tiles(ctypes.byref(p), 0, 0, None, None, 1) == dt.DT_ERR_INVALID
     assert lib.dt_key_set_tiles(ctypes.byref(p), 0, 0, None, None, 0) == 2
+
+
+@pytest.mark.parametrize("wi", range(len(wl.WORKLOADS)))
+def test_share_counts_match_oracle_counts(wi):
+    """Attention sharing counts from libdt: across CFG branches half of the
+    plan's computed blocks and FLOPs (the conditional half) with every other
+    block skipped; across timesteps nothing computed and every block of every
+    head skipped (the blocks an all-compute plan computes, by the oracle)."""
+    w = wl.WORKLOADS[wi]
+    H = 2 * w.H
+    win = bool(w.window)
+    mode = orc.MODE_WINDOW if win else orc.MODE_PROXIMITY
+    P = 1 if win else w.P
+    r = 0 if win else w.P // 2
+    _, full, _ = orc.build_plan(orc.MODE_ALL_COMPUTE if not win else orc.MODE_WINDOW, H, w.S, w.D, P, 1,
+                                window=w.window)
+    p1 = dt.params(H, w.S, w.D, P, mode, r, w.window, 1)
+    _, c1 = dt.dt_plan_build(p1)
+    assert dt.dt_plan_share_counts(p1, dt.DT_SHARE_TIMESTEP) == {
+        "computed_blocks": 0, "skipped_blocks": full["computed_blocks"] + full["skipped_blocks"], "computed_flops": 0}
+    st = np.full(dt.dt_plan_geometry(p1), 1, dtype=np.int32)
+    p2 = dt.params(H, w.S, w.D, P, mode, r, w.window, 2)
+    _, c2 = dt.dt_plan_build(p2, st)
+    for c in (c1, c2):
+        _, ch, _ = orc.build_plan(mode, H // 2, w.S, w.D, P, 2 if c is c2 else 1, r=r, window=w.window,
+                                  stamps=np.ones_like(st) if c is c2 else None)
+        got = dt.dt_plan_share_counts(p1, dt.DT_SHARE_CFG, c)
+        assert got["computed_blocks"] == ch["computed_blocks"]
+        assert got["computed_flops"] == ch["computed_flops"]
+        assert got["computed_blocks"] + got["skipped_blocks"] == c["computed_blocks"] + c["skipped_blocks"]
+
+
+def test_share_calls_validated_on_the_host():
+    import ctypes
+    lib = dt.load()
+    p = dt.params(3, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1)
+    io = dt.Plan()
+    assert lib.dt_plan_share_counts(ctypes.byref(p), dt.DT_SHARE_CFG, ctypes.byref(io)) == dt.DT_ERR_INVALID  # odd H
+    p.H = 4
+    assert lib.dt_plan_share_counts(ctypes.byref(p), 7, ctypes.byref(io)) == dt.DT_ERR_INVALID
+    assert lib.dt_plan_share_counts(ctypes.byref(p), dt.DT_SHARE_CFG, None) == dt.DT_ERR_INVALID
+    p.H = 3
+    assert lib.dt_attn_cfg_shared(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_INVALID
+    p.H = 4
+    assert lib.dt_attn_cfg_shared(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_INVALID   # null buffers

@@ -133,6 +133,17 @@ def test_video_workload_full_size_sampled_rows():
                            rows=sample_rows(w.S, w.P, n_extra=24))
 
 
+
+def test_video_workload_benchmark_configuration():
+    """The configuration bench.py times: the full-size video workload, an
+    anchor step, then two 50%-reuse steps (8 of 16 partitions reused), on
+    sampled heads and rows, including the fresh cache slots."""
+    w = wl.WORKLOADS[3]
+    sched = [(1, dt.DT_MODE_PROXIMITY, 8, None), (2, dt.DT_MODE_PROXIMITY, 8, None),
+             (3, dt.DT_MODE_PROXIMITY, 8, None)]
+    run_partition_schedule(w.H, w.S, w.D, w.P, sched, wl.stream_for(w).next_step, heads=[0, 21, 39],
+                           rows=sample_rows(w.S, w.P, n_extra=24))
+
 # ------------------------------------------------------------------ edge cases
 
 @pytest.mark.parametrize("H,S,D,P,r", [
@@ -157,6 +168,29 @@ def test_stress_inputs(kind, D):
     q, k, v = wl.stress_inputs(H, S, D, kind, seed=D)
     run_partition_schedule(H, S, D, P, [(1, dt.DT_MODE_ALL_COMPUTE, 0, None)], lambda: (q, k, v),
                            output_scaled=True)
+
+
+def perturbed(bits, sigma, seed):
+    """bf16 inputs plus sigma * N(0,1), rounded back to bf16 (a later step of
+    a stress set)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = wl.bf16_bits_to_f32(bits) + np.float32(sigma) * rng.standard_normal(bits.shape, dtype=np.float32)
+    return wl.f32_to_bf16_bits(x)
+
+
+@pytest.mark.parametrize("kind", ["unit", "spiky"])
+@pytest.mark.parametrize("D,g", [(64, 0), (72, 0), (128, 0), (128, 2)])
+def test_stress_inputs_through_reuse(kind, D, g):
+    """Stress sets through an anchor and then reuse steps: cached states with
+    a large spread of LSEs (logits above 20 in "spiky") are composed with
+    fresh ones by the epilogue's reuse merge."""
+    H, S, P = 2, 1500, 6
+    q, k, v = wl.stress_inputs(H, S, D, kind, seed=D + 1)
+    steps = [(q, k, v)] + [tuple(perturbed(x, 0.05, 10 * t + j) for j, x in enumerate((q, k, v))) for t in (1, 2)]
+    it = iter(steps)
+    sched = [(1, dt.DT_MODE_PROXIMITY, 2, None), (2, dt.DT_MODE_PROXIMITY, 2, None),
+             (3, dt.DT_MODE_PROXIMITY, 1 if g else 4, None)]
+    run_partition_schedule(H, S, D, P, sched, lambda: next(it), output_scaled=True, group=g, check_untouched=True)
 
 
 def test_all_reuse_reproduces_previous_output_and_explicit_plan():
@@ -222,10 +256,79 @@ def test_window_small(H, S, D, W):
 
 
 def test_window_workload_full_size_sampled_rows():
+    """The full-size window workload over its whole schedule: the anchor step
+    (full attention, R made) and the three window + residual steps."""
     w = wl.WORKLOADS[4]
     rows = np.unique(np.concatenate([np.arange(0, 130), np.arange(w.S - 130, w.S),
                                      np.random.Generator(np.random.PCG64(3)).choice(w.S, 60, replace=False)]))
-    run_window_schedule(w.H, w.S, w.D, w.window, 2, wl.stream_for(w).next_step, heads=[0, 15], rows=rows)
+    run_window_schedule(w.H, w.S, w.D, w.window, w.steps, wl.stream_for(w).next_step, heads=[0, 15], rows=rows)
+
+
+def run_window_abi(H, S, D, W, steps, inputs, fill=float("nan")):
+    """Window mode through the C ABI directly, with caller buffers that start
+    filled with `fill` (NaN by default): every row of R must be written at the
+    anchor step, whatever the caller's buffer held."""
+    dev = "cuda"
+    R = torch.full((H, S, D), fill, dtype=torch.float32, device=dev)
+    O = torch.full((H, S, D), fill, dtype=torch.bfloat16, device=dev)
+    L = torch.full((H, S), fill, dtype=torch.float32, device=dev)
+    Qd, Kd, Vd = (torch.empty((H, S, D), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    counters = torch.zeros(4, dtype=torch.int64, device=dev)
+    status = torch.zeros(4, dtype=torch.int32, device=dev)
+    Rref = {}
+    stamps = None
+    for step in range(1, steps + 1):
+        q, k, v = inputs()
+        for dst, src in ((Qd, q), (Kd, k), (Vd, v)):
+            dst.copy_(torch.from_numpy(src.view(np.int16)).view(torch.bfloat16))
+        p = dt.params(H, S, D, 1, dt.DT_MODE_WINDOW, 0, W, step)
+        if stamps is None:
+            stamps = np.full(dt.dt_plan_geometry(p), -1, dtype=np.int32)
+        plan, counts = dt.dt_plan_build(p, stamps)
+        d_plan = torch.from_numpy(plan).to(dev)
+        counters.zero_()
+        dt.dt_attn_partial_fused(p, d_plan, Qd, Kd, Vd, None, None, R, O, L, counters, status)
+        torch.cuda.synchronize()
+        assert int(status[0]) == 0, dt.dt_status_string(int(status[0]))
+        c = counters.cpu().numpy()
+        assert int(c[0]) == counts["computed_blocks"] and int(c[1]) == counts["skipped_blocks"]
+        O_ref, L_ref = orc.window_step(q, k, v, W, step == 1, Rref)
+        if step == 1:
+            R_ref = np.stack([np.stack([Rref[(h, r)] for r in range(S)]) for h in range(H)])
+            check_out(to_np(R), R_ref, "R", max_abs=1e-2, rel=1e-2)
+        check_out(to_np(O), O_ref, f"O step {step}")
+        check_lse(to_np(L), L_ref, f"LSE step {step}")
+
+
+@pytest.mark.parametrize("H,S,D,W", [
+    (2, 200, 128, 400),      # W >= 2S: every key in every window, R = 0 everywhere
+    (1, 2000, 72, 1900),     # interior query tiles whose band covers all keys (empty complement)
+    (1, 2000, 64, 1900),
+    (2, 1000, 128, 100),     # ordinary band: every row has a complement
+])
+def test_window_residual_written_for_every_row(H, S, D, W):
+    run_window_abi(H, S, D, W, 3, stream_of(H, S, D, 0.03, seed=S + W))
+
+
+@pytest.mark.parametrize("D", [72, 128])
+def test_window_spiky_inputs(D):
+    """Window mode on the spiky stress set: the residual of rows whose large
+    logits fall outside the band is large, and later steps add it back."""
+    H, S, W = 2, 1200, 256
+    q, k, v = wl.stress_inputs(H, S, D, "spiky", seed=D + 5)
+    steps = iter([(q, k, v)] + [tuple(perturbed(x, 0.05, 20 * t + j) for j, x in enumerate((q, k, v)))
+                                for t in (1, 2)])
+    sess = Session(H, S, D, 1, mode=dt.DT_MODE_WINDOW, window=W)
+    sess.R.fill_(float("nan"))
+    R = {}
+    for step in (1, 2, 3):
+        qq, kk, vv = next(steps)
+        sess.set_inputs(qq, kk, vv)
+        sess.step(step)
+        sess.check()
+        O_ref, L_ref = orc.window_step(qq, kk, vv, W, step == 1, R)
+        check_out(to_np(sess.O), O_ref, f"O step {step}", output_scaled=True)
+        check_lse(to_np(sess.L), L_ref, f"LSE step {step}")
 
 
 @pytest.mark.gpu
@@ -435,17 +538,20 @@ def test_importance_weights_and_plan_match_oracle(H, S, D, P, g):
 
 # ------------------------------------------------------- attention sharing
 
-@pytest.mark.parametrize("g", [0, 2])
-def test_cfg_shared_step(g):
+@pytest.mark.parametrize("g,sd", [(0, 0), (2, 0), (0, 1)])
+def test_cfg_shared_step(g, sd):
     """Sharing across CFG branches: heads [0, H/2) (conditional) are computed
     and match the oracle on their own inputs; heads [H/2, H) receive the same
-    bytes, their inputs are ignored and their cache slots stay untouched."""
+    output bytes, their inputs are ignored, and the states the conditional
+    heads computed become theirs too (same cache bytes).  A later ordinary
+    step on both halves then reuses those states and matches the oracle on
+    every head."""
     Hb, S, D, P = 2, 1024, 64, 4
     r = 1
     cond = wl.InputStream(Hb, S, D, 0.05, seed=90)
     other = wl.InputStream(Hb, S, D, 0.5, seed=91)
-    sess = Session(2 * Hb, S, D, P, reuse_per_row=r, group=g)
-    cache = orc.StateCache()
+    sess = Session(2 * Hb, S, D, P, reuse_per_row=r, group=g, state_dtype=sd)
+    cache = orc.StateCache(bf16=sd == dt.DT_STATE_BF16)
     for step in (1, 2):
         qc, kc, vc = cond.next_step()
         qu, ku, vu = other.next_step()
@@ -453,16 +559,61 @@ def test_cfg_shared_step(g):
         sess.counters.zero_()
         counts = sess.step_cfg_shared(step)
         sess.check()
-        O_ref, L_ref, _ = orc.partition_step(qc, kc, vc, sess.last_plan, S, P, cache, group=g)
+        O_ref, L_ref, fresh = orc.partition_step(qc, kc, vc, sess.last_plan, S, P, cache, group=g)
+        for (kk, h), items in fresh.items():       # the unconditional heads take the conditional states
+            for rs, (o_f, l_f) in items:
+                cache.put(kk, h + Hb, rs, o_f, l_f)
         check_out(to_np(sess.O[:Hb]), O_ref, f"cond O step {step}")
         check_lse(to_np(sess.L[:Hb]), L_ref, f"cond LSE step {step}")
         assert torch.equal(sess.O[Hb:].view(torch.int16), sess.O[:Hb].view(torch.int16))
         assert torch.equal(sess.L[Hb:], sess.L[:Hb])
-        assert torch.all(sess.cache_O[:, Hb:] == 0) and torch.all(torch.isneginf(sess.cache_L[:, Hb:]))
+        view = (lambda t: t.view(torch.int16)) if sd else (lambda t: t)
+        assert torch.equal(view(sess.cache_O[:, Hb:]), view(sess.cache_O[:, :Hb]))
+        assert torch.equal(sess.cache_L[:, Hb:], sess.cache_L[:, :Hb])
         c = sess.counters.cpu().numpy()
         assert int(c[0]) == counts["computed_blocks"]
         assert counts["computed_blocks"] + counts["skipped_blocks"] == \
             2 * Hb * sum(orc.n_kv_tiles(a, b) for a, b in orc.partitions(S, P)) * len(orc.query_tiles(S, P))
+    # an ordinary step on both branches reuses the shared states
+    qc, kc, vc = cond.next_step()
+    qu, ku, vu = other.next_step()
+    q, k, v = (np.concatenate([a, b]) for a, b in ((qc, qu), (kc, ku), (vc, vu)))
+    sess.set_inputs(q, k, v)
+    sess.step(3)
+    sess.check()
+    O_ref, L_ref, _ = orc.partition_step(q, k, v, sess.last_plan, S, P, cache, group=g)
+    assert (sess.last_plan == orc.REUSE).any()
+    check_out(to_np(sess.O), O_ref, "both branches O step 3")
+    check_lse(to_np(sess.L), L_ref, "both branches LSE step 3")
+
+
+def test_cfg_shared_window_mode():
+    """CFG sharing in window mode: the residual made at the anchor by the
+    conditional heads is the unconditional heads' residual too, so a later
+    ordinary window step matches the oracle on every head."""
+    Hb, S, D, W = 2, 1000, 72, 256
+    cond = wl.InputStream(Hb, S, D, 0.03, seed=92)
+    other = wl.InputStream(Hb, S, D, 0.5, seed=93)
+    sess = Session(2 * Hb, S, D, 1, mode=dt.DT_MODE_WINDOW, window=W)
+    sess.R.fill_(float("nan"))
+    R = {}
+    qc, kc, vc = cond.next_step()
+    qu, ku, vu = other.next_step()
+    sess.set_inputs(*(np.concatenate([a, b]) for a, b in ((qc, qu), (kc, ku), (vc, vu))))
+    sess.step_cfg_shared(1)
+    sess.check()
+    O_ref, L_ref = orc.window_step(qc, kc, vc, W, True, R)
+    for (h, row), val in list(R.items()):
+        R[(h + Hb, row)] = val
+    check_out(to_np(sess.O[:Hb]), O_ref, "cond O anchor")
+    assert torch.equal(sess.R[Hb:], sess.R[:Hb])
+    q, k, v = (np.concatenate([a, b]) for a, b in zip(cond.next_step(), other.next_step()))
+    sess.set_inputs(q, k, v)
+    sess.step(2)
+    sess.check()
+    O_ref, L_ref = orc.window_step(q, k, v, W, False, R)
+    check_out(to_np(sess.O), O_ref, "both branches O step 2")
+    check_lse(to_np(sess.L), L_ref, "both branches LSE step 2")
 
 
 def test_share_previous_output():
