@@ -36,6 +36,7 @@ import numpy as np  # noqa: E402
 
 METRIC = "attention ms/denoise-step & TFLOP/s on computed blocks vs B200 bf16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+NOMINAL_BF16_TFLOPS = 2250.0      # B200 dense bf16, nominal (context for the measured-peak fraction)
 
 
 def parse_args():
@@ -56,6 +57,8 @@ def parse_args():
     ap.add_argument("--heads", type=int, default=None, help="override H (smaller profiling captures)")
     ap.add_argument("--group", type=int, default=0,
                     help="state grouping: groups of G adjacent partitions, --reuse then counts groups")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (tiny, DiT-XL/2-like, PixArt-like, window)")
     ap.add_argument("--no-grouped", action="store_true",
                     help="skip the grouped-cache, compose, bf16-cache and importance measurements")
     return ap.parse_args()
@@ -92,7 +95,7 @@ def job_throughput(flops_per_rank, world, ms):
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for fn in ("attn_fused_sm100.cu", "sm100.cuh", "geometry.h", "attn_fused.h", "exp2_poly.h"):
+    for fn in ("attn_fused_sm100.cu", "sm100.cuh", "geometry.h", "attn_fused.h"):
         with open(os.path.join(ROOT, "partitioned_attention_state_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -223,6 +226,46 @@ def oracle_sample(w, r, budget_s=12.0, heads=(0,), inputs=None, group=0):
                       f"{layout} ({flops / 1e9:.1f} GFLOP, {elapsed:.1f} s), float64 numpy oracle"}
 
 
+def oracle_sample_window(w, budget_s=4.0, inputs=None):
+    """Time the CPU oracle on a bounded sample of one window + residual step
+    (steps >= 2): whole query tiles of one head, their window attention plus
+    the residual add; the residual comes from an untimed anchor on the same
+    rows."""
+    import oracle as orc
+    from partitioned_attention_state_b200 import workloads as wl
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    if inputs is None:
+        s = wl.InputStream(w.H, w.S, w.D, w.sigma, seed=w.seed)
+        inputs = s.next_step() + s.next_step()
+    q1, k1, v1, q2, k2, v2 = inputs
+    Q1, K1, V1 = (orc.widen_bf16(x[[0]]) for x in (q1, k1, v1))
+    Q2, K2, V2 = (orc.widen_bf16(x[[0]]) for x in (q2, k2, v2))
+    tiles = orc.query_tiles(w.S, 1, window=w.window)
+    order = np.random.Generator(np.random.PCG64(7)).permutation(len(tiles))
+    hw = w.window // 2
+    flops = elapsed = 0.0
+    n_tiles = 0
+    for t in order:
+        _, q0, qe = tiles[t]
+        rows = np.arange(q0, qe)
+        R = {}
+        orc.window_step(Q1, K1, V1, w.window, True, R, rows=rows)          # anchor (untimed)
+        t0 = time.perf_counter()
+        orc.window_step(Q2, K2, V2, w.window, False, R, rows=rows)
+        elapsed += time.perf_counter() - t0
+        flops += 4 * w.D * sum(min(w.S - 1, i + hw) - max(0, i - hw) + 1 for i in range(q0, qe))
+        n_tiles += 1
+        if elapsed >= budget_s:
+            break
+    return {"tflops": flops / elapsed / 1e12, "threads": threads,
+            "sample": f"{n_tiles} query tiles x 1 head of one window + residual step "
+                      f"({flops / 1e9:.2f} GFLOP, {elapsed:.1f} s), float64 numpy oracle"}
+
+
 def run_reference(args, w, r, rank, group=0):
     if rank != 0:
         return
@@ -349,7 +392,15 @@ def main():
                 "reuse_per_row": rr, "ms_per_step": ms, "kernel_ms": km,
                 "tflops": c["computed_flops"] / (km * 1e-3) / 1e12,
                 "frac_of_peak": c["computed_flops"] / (km * 1e-3) / 1e12 / peak_tf,
+                "frac_of_nominal": c["computed_flops"] / (km * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS,
+                "ms_over_ms_r0": None,
                 "computed_blocks": c["computed_blocks"], "skipped_blocks": c["skipped_blocks"]}
+        # "time falls in proportion to reuse": ms(r)/ms(0) beside the computed-FLOP fraction
+        base = sweep.get("0%")
+        if base:
+            for e in sweep.values():
+                e["ms_over_ms_r0"] = e["kernel_ms"] / base["kernel_ms"]
+                e["computed_fraction"] = e["computed_blocks"] / max(1, base["computed_blocks"])
         sess.r = r
 
     # standalone state merge over the whole cache (HBM-bound)
@@ -482,6 +533,57 @@ def main():
                    "GB/s": cbytes / (cms * 1e-3) / 1e9, "frac_of_hbm": cbytes / (cms * 1e-3) / 1e9 / hbm}
         del gs
 
+    # every other workload of the hot-path table, timed like the headline
+    # (anchor step, then graph replays of the reuse step), with the CPU
+    # oracle on a bounded sample of each
+    configs = None
+    if not args.no_configs and args.heads is None:
+        configs = {}
+        for ow in wl.WORKLOADS:
+            if ow.name == w.name:
+                continue
+            owin = ow.mode == "window"
+            for orr in (ow.reuse if not owin else (0,)):
+                cs = Session(ow.H, ow.S, ow.D, ow.P, mode=dt.DT_MODE_WINDOW if owin else dt.DT_MODE_PROXIMITY,
+                             reuse_per_row=orr, window=ow.window)
+                ostream = wl.stream_for(ow)
+                oq1 = ostream.next_step()
+                oq2 = ostream.next_step()
+                cs.set_inputs(*oq1)
+                cs.step(1)
+                cs.set_inputs(*oq2)
+                cs.check()
+                graph = cs.capture_step(2)
+                for _ in range(args.warmup):
+                    graph.replay()
+                barrier()
+                nrep = max(10, args.steps)
+                evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(nrep)]
+                for a_, b_ in evs:
+                    a_.record(cur)
+                    oc = graph.replay()
+                    b_.record(cur)
+                barrier()
+                cs.check()
+                kms = max_over_ranks([float(np.median([a_.elapsed_time(b_) for a_, b_ in evs]))], "cuda")[0]
+                tf = oc["computed_flops"] / (kms * 1e-3) / 1e12
+                entry = {"reuse_per_row": orr, "ms_per_step": kms, "tflops": tf, "frac": tf / peak_tf,
+                         "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS,
+                         "reuse_ratio": oc["skipped_blocks"] / max(1, oc["skipped_blocks"] + oc["computed_blocks"]),
+                         "computed_flops": oc["computed_flops"], "computed_blocks": oc["computed_blocks"],
+                         "skipped_blocks": oc["skipped_blocks"],
+                         "timing": "median of per-launch CUDA events over graph replays"}
+                del graph, cs
+                torch.cuda.empty_cache()
+                if rank == 0 and not args.no_cpu:
+                    if owin:
+                        res = oracle_sample_window(ow, budget_s=3.0, inputs=oq1 + oq2)
+                    else:
+                        res = oracle_sample(ow, orr, budget_s=3.0, inputs=oq1 + oq2)
+                    entry["cpu_oracle"] = {"tflops": res["tflops"], "cores": res["threads"], "sample": res["sample"]}
+                configs[f"{ow.name}" + (f" r={orr}" if len(ow.reuse) > 1 else "")] = entry
+
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -532,13 +634,15 @@ def main():
                        "l2": "inputs larger than L2 (no flush): Q/K/V and the state cache exceed 126 MB"},
             "roofline": {"bound": "tensor", "kernel": "attn_partial_fused_kernel", "achieved": achieved,
                          "peak": peak_tf, "peak_kind": f"{pk_kind} bf16 dense (burst)", "unit": "TFLOP/s",
-                         "frac": achieved / peak_tf, "traffic": traffic, "kernel_ms": kern_ms,
+                         "frac": achieved / peak_tf, "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
+                         "nominal_peak": NOMINAL_BF16_TFLOPS, "traffic": traffic, "kernel_ms": kern_ms,
                          "flops_per_launch": flops},
             "gpu_launches": args.steps,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
             "reuse_sweep": sweep,
+            "configs": configs,
             "state_merge": merge,
             "grouped": grouped,
             "group_compose": compose,

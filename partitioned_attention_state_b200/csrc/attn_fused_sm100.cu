@@ -67,7 +67,6 @@
 
 #include "../../include/dt.h"
 #include "attn_fused.h"
-#include "exp2_poly.h"
 #include "geometry.h"
 #include "sm100.cuh"
 
@@ -129,10 +128,6 @@ struct Cfg {
   static constexpr int kSmem = kTileBytes * (1 + 2 * kStages) + kOtotBytes + kStatsBytes + kNumBars * 8 + 16;
   static_assert(kSmem <= 232448, "shared memory budget");
 };
-
-// Exponentials of an unmasked tile: when kEmuMod > 0 every kEmuMod-th
-// repetition (4 values) is evaluated on the FMA pipe instead of MUFU.
-constexpr int kEmuMod = 0;
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
@@ -603,9 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               float x0, x1, x2, x3;
               upk2(fma2(pk2(u2f(sr[e]), u2f(sr[e + 1])), sl2x2, nma), x0, x1);
               upk2(fma2(pk2(u2f(sr[e + 2]), u2f(sr[e + 3])), sl2x2, nmb), x2, x3);
-              const bool emu = kEmuMod > 0 && !masked && !precise && (r4 % (kEmuMod > 0 ? kEmuMod : 1)) == kEmuMod - 1;
-              const float p0 = emu ? dt_exp2_fma(x0) : ex2(x0), p1 = emu ? dt_exp2_fma(x1) : ex2(x1);
-              const float p2 = emu ? dt_exp2_fma(x2) : ex2(x2), p3 = emu ? dt_exp2_fma(x3) : ex2(x3);
+              const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
               la[r4 & 1] = add2(la[r4 & 1], pk2(p0, p1));
               lb[r4 & 1] = add2(lb[r4 & 1], pk2(p2, p3));
               ph[2 * r4] = pack_bf16x2(p0, p1);

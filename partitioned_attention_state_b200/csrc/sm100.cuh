@@ -35,18 +35,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Non-blocking probe: has the phase of `parity` completed?
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -60,9 +48,6 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-#ifndef DT_WAIT_MODE
-#define DT_WAIT_MODE 1
-#endif
 // try_wait with a suspend-time hint (ns): the thread sleeps until the phase
 // completes or the hint elapses, instead of re-polling.
 __device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
@@ -82,19 +67,7 @@ __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, v
                                             int32_t code, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer();
   while (true) {
-#if DT_WAIT_MODE == 1
     if (mbar_try_wait_hint(bar, parity, 200000u)) return true;
-#elif DT_WAIT_MODE == 2
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
-      if (mbar_try_wait(bar, parity)) return true;
-      __nanosleep(32);
-    }
-#else
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-#endif
     if (*abort) return false;
     if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
