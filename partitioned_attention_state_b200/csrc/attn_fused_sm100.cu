@@ -118,7 +118,7 @@ struct Cfg {
   static constexpr int kColS = 0;
   static constexpr int kColOpart = 128 * kNS;
   static_assert(kColOpart + DP <= 512, "tensor memory budget");
-  static constexpr int kOtotBytes = DP * 128 * 4;      // O_tot in shared memory, column-major [DP][128] fp32
+  static constexpr int kOtotBytes = DP * 128 * 4;      // O_tot in shared memory, [128][DP] fp32 (swizzled)
   // barrier indices
   static constexpr int bQFull = 0, bQEmpty = 1, bKFull = 2, bVFull = 2 + kStages, bKEmpty = 2 + 2 * kStages,
                        bVEmpty = 2 + 3 * kStages, bSFull = 2 + 4 * kStages, bPFull = bSFull + kNS,
@@ -203,6 +203,18 @@ __device__ __forceinline__ int visit_tile(const KeySet& ks, int nt, int off, int
   return ks.tile(k >= nt ? k - nt : k);
 }
 
+// O_tot (the running composition of an item's states, fp32, shared memory):
+// row-major [128][DP], its 16-byte chunks XOR-swizzled by (row & 7) inside
+// each full group of 8 chunks.  A warp touching one chunk of 32 rows (a row
+// per lane) or all chunks of one row (a chunk per lane) then hits every bank
+// once per 8-lane phase of a 16-byte access.
+template <int DP>
+__device__ __forceinline__ float4* ot_chunk(float* sO, int row, int cc) {
+  constexpr int kChunks = DP / 4;
+  const int sw = ((cc | 7) < kChunks) ? (cc ^ (row & 7)) : cc;
+  return reinterpret_cast<float4*>(sO + row * DP + 4 * sw);
+}
+
 // Issue O_part += P V for tile g (P read from tensor memory, V from the ring).
 template <int DP>
 __device__ __forceinline__ bool issue_pv(uint64_t* bars, uint32_t tmem, uint32_t aV, uint32_t g, uint32_t seg,
@@ -264,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
   uint8_t* sQ = smem;
   uint8_t* sK = smem + C::kTileBytes;
   uint8_t* sV = sK + C::kStages * C::kTileBytes;
-  float* sO = reinterpret_cast<float*>(sV + C::kStages * C::kTileBytes);       // O_tot [DP][128]
+  float* sO = reinterpret_cast<float*>(sV + C::kStages * C::kTileBytes);       // O_tot [128][DP]
   float* stat_m = sO + DP * 128;                                               // [2][128]
   float* stat_l = stat_m + 256;                                                // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(stat_l + 256);
@@ -661,10 +673,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t opart = tmem + lane_base + C::kColOpart;
     constexpr int D = DP == 80 ? 72 : DP;   // head dims 64, 72, 128 (padded 64, 80, 128)
-    // O_tot of this thread's row lives in shared memory, column-major
-    // ([column][row]: consecutive threads, consecutive banks), unnormalised
-    // relative to m_tot.  Only this thread touches its row.
-    float* orow = sO + r;
+    // O_tot rows are unnormalised relative to m_tot.  A thread owns its row
+    // (fresh states, output); the reuse merge updates the warp's 32 rows
+    // cooperatively, one row per load instruction.
     uint32_t cseg = 0;
     uint32_t n_comp = 0, n_skip = 0, n_fresh = 0, n_read = 0;
     for (int idx = p.item0 + blockIdx.x; idx < p.item_end; idx += gridDim.x) {
@@ -678,11 +689,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       bool have = false, use_r = false;
       // O_tot starts at zero, so the merges below need no separate first-state case
 #pragma unroll 4
-      for (int c = 0; c < DP; ++c) orow[c * 128] = 0.f;
+      for (int cc = 0; cc < DP / 4; ++cc) *ot_chunk<DP>(sO, r, cc) = make_float4(0.f, 0.f, 0.f, 0.f);
+      __syncwarp();
       // Cached states of the REUSE pairs are composed into O_tot interleaved
-      // with the fresh ones, a fixed share before each fresh state (their
-      // loads are latency-bound; composing them all first would hold up the
-      // release of O_part that the MMA warps wait on).  The order depends
+      // with the fresh ones, a fixed share after each fresh state, once its
+      // O_part is back with the MMA warps (their loads are latency-bound;
+      // composing them before a fresh state would hold up the release of
+      // O_part that the next key set's PV waits on).  The order depends
       // only on the plan, so results are reproducible run to run.  jr walks
       // the key sets in visiting order; merged counts reused sets done.
       const int sets_fresh = __popcll(cm), sets_reused = G.P - sets_fresh;
@@ -706,38 +719,46 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             b = nonempty ? ex2(m_c - m_new) : 0.f;
           }
           const float l_new = a * l_tot + b;
-          const float4* src = reinterpret_cast<const float4*>(p.cache_O + slot * D);
-          const uint4* srch = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.cache_O) + slot * D);
-          const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          // The warp's 32 slot rows are contiguous: lane l reads 16 bytes (8
+          // of bf16) of every row, so each load instruction covers one whole
+          // row; 16 rows are in flight together.  Rows the slot has no state
+          // for (ragged tile, empty state) are not read.
+          const uint32_t live = __ballot_sync(0xffffffffu, valid && nonempty);
+          __syncwarp();                                   // the lanes' own-row writes are visible
+          const size_t row0 = slot - r + 32 * q4;           // slot row of the warp's first row
+          const bool lane_on = 4 * lane < D;
 #pragma unroll 1
-          for (int c1 = 0; c1 < D; c1 += 32) {             // 32 cached columns in flight together
-            float4 cv[8];
-            if (CBF) {                                     // bf16 OUT: 8 columns per 16-byte load
-              uint4 hv[4];
+          for (int i0 = 0; i0 < 32; i0 += 16) {
+            float4 cv[16];
 #pragma unroll
-              for (int c = 0; c < 4; ++c)
-                hv[c] = (c1 + 8 * c < D && valid && nonempty) ? __ldcs(srch + c1 / 8 + c) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                cv[2 * c] = make_float4(bf16lo(hv[c].x), bf16hi(hv[c].x), bf16lo(hv[c].y), bf16hi(hv[c].y));
-                cv[2 * c + 1] = make_float4(bf16lo(hv[c].z), bf16hi(hv[c].z), bf16lo(hv[c].w), bf16hi(hv[c].w));
+            for (int k = 0; k < 16; ++k) {
+              const bool on = lane_on && ((live >> (i0 + k)) & 1u);
+              if (CBF) {
+                const uint2 hv = on ? __ldcs(reinterpret_cast<const uint2*>(
+                                          reinterpret_cast<const __nv_bfloat16*>(p.cache_O) + (row0 + i0 + k) * D) + lane)
+                                    : make_uint2(0, 0);
+                cv[k] = make_float4(bf16lo(hv.x), bf16hi(hv.x), bf16lo(hv.y), bf16hi(hv.y));
+              } else {
+                cv[k] = on ? __ldcs(reinterpret_cast<const float4*>(p.cache_O + (row0 + i0 + k) * D) + lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
               }
-            } else {
-#pragma unroll
-              for (int c = 0; c < 8; ++c)
-                cv[c] = (c1 + 4 * c < D && valid && nonempty) ? __ldcs(src + c1 / 4 + c) : z4;
             }
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              if (c1 + 4 * c < D) {
-                float* o = orow + (c1 + 4 * c) * 128;
-                o[0] = fmaf(a, o[0], b * cv[c].x);
-                o[128] = fmaf(a, o[128], b * cv[c].y);
-                o[256] = fmaf(a, o[256], b * cv[c].z);
-                o[384] = fmaf(a, o[384], b * cv[c].w);
+            for (int k = 0; k < 16; ++k) {
+              const int row = 32 * q4 + i0 + k;
+              const float ak = __shfl_sync(0xffffffffu, a, i0 + k), bk = __shfl_sync(0xffffffffu, b, i0 + k);
+              if (lane_on) {
+                float4* o = ot_chunk<DP>(sO, row, lane);
+                float4 ov = *o;
+                ov.x = fmaf(ak, ov.x, bk * cv[k].x);
+                ov.y = fmaf(ak, ov.y, bk * cv[k].y);
+                ov.z = fmaf(ak, ov.z, bk * cv[k].z);
+                ov.w = fmaf(ak, ov.w, bk * cv[k].w);
+                *o = ov;
               }
             }
           }
+          __syncwarp();
           if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
           have = have || nonempty;
           ++jr;
@@ -774,7 +795,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         }
         const uint32_t st = cseg & 1;
         ++fi;
-        while (jr < G.P && merged * sets_fresh < fi * sets_reused) merge_next_reused();
         if (!warp_wait(&bars[C::bStFull + st], (cseg >> 1) & 1, abort_flag, p.status, lim)) goto ep_done;
         const float m_s = stat_m[st * 128 + r], l_s = stat_l[st * 128 + r];
         mbar_arrive(&bars[C::bStFree + st]);
@@ -804,13 +824,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
 #pragma unroll
         for (int c = 0; c < D; c += 4) {
           float old[4], nw[4], x[4];
+          float4* oc = ot_chunk<DP>(sO, r, c / 4);
+          const float4 ov = *oc;
+          old[0] = ov.x; old[1] = ov.y; old[2] = ov.z; old[3] = ov.w;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            old[k] = orow[(c + k) * 128];
             x[k] = u2f(op[c + k]);
             nw[k] = fmaf(a, old[k], b * x[k]);
-            orow[(c + k) * 128] = nw[k];
           }
+          *oc = make_float4(nw[0], nw[1], nw[2], nw[3]);
           if (valid) {
             if (!WIN && CBF) {
               uint2 pk;
@@ -834,6 +856,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
         have = have || nonempty;
         ++cseg;
+        // this fresh state's share of the cached states, composed while the
+        // MMA warps compute the next key set (O_part is already released)
+        while (jr < G.P && merged * sets_fresh < fi * sets_reused) merge_next_reused();
       }
       while (jr < G.P) merge_next_reused();
       // final: O = O_tot / l_tot (+ R), LSE = m_tot + log2(l_tot), in natural units
@@ -843,8 +868,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const float* rr = p.R + ((size_t)h * G.S + qrow) * D;
 #pragma unroll 2
         for (int c = 0; c < D; c += 4) {
-          float v0 = orow[c * 128] * inv, v1 = orow[(c + 1) * 128] * inv;
-          float v2 = orow[(c + 2) * 128] * inv, v3 = orow[(c + 3) * 128] * inv;
+          const float4 ov = *ot_chunk<DP>(sO, r, c / 4);
+          float v0 = ov.x * inv, v1 = ov.y * inv, v2 = ov.z * inv, v3 = ov.w * inv;
           if (use_r) {
             const float4 rv = __ldcs(reinterpret_cast<const float4*>(rr + c));
             v0 += rv.x; v1 += rv.y; v2 += rv.z; v3 += rv.w;
