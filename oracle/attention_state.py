@@ -46,6 +46,21 @@ notes of the repository):
     smallest ASE, never the local set nor a never-written slot, lower index
     first among equal values, the products taken in float32 as the GPU-side
     weights are float32;
+  * anchor-guided planning (the selection strategy's anchor condition, scale
+    ratios and adapted threshold; equations lost): the state error of a key
+    set k computed at step t is the relative difference ||OUT_t - OUT_c|| /
+    ||OUT_t|| (Frobenius, over the tile's rows and all heads) between the
+    fresh OUT and the OUT its cache slot held; the local drift of a tile is
+    the state error of its own set (computed every step); an anchor is
+    taken at step 1 and when the local drift accumulated since the last
+    anchor exceeds a budget theta for any tile (replacing a static maximum
+    age); at an anchor the scale ratio of every other set with a previous
+    state is its state error per step of cache age, alpha = e / (t - t_c)
+    (linear growth with age), and the threshold epsilon is the rho-quantile
+    of the global importance-weighted rates w * alpha over all (tile, set)
+    pairs (rho the target reuse ratio); between anchors a set is reused iff
+    w * alpha * (t - t_c) <= epsilon (float32 products), never the local set
+    nor a never-written slot; before the first measured anchor alpha = 1;
   * Dynamic Group State Compose by a factor k: the new group i is old groups
     k i .. k i + k - 1, its cached state their composition, its stamp the
     oldest of theirs (never written if any was never written).
@@ -68,6 +83,7 @@ MODE_ALL_REUSE = 2
 MODE_EXPLICIT = 3
 MODE_WINDOW = 4
 MODE_IMPORTANCE = 5
+MODE_ANCHOR = 6
 
 __all__ = [
     "TILE", "REUSE", "COMPUTE", "MODE_ALL_COMPUTE", "MODE_PROXIMITY",
@@ -78,6 +94,7 @@ __all__ = [
     "partition_step", "window_step", "softmax_scale",
     "n_groups", "group_key_sets", "group_proximity_row", "key_sets_of_tile",
     "compose_groups", "MODE_IMPORTANCE", "state_importance", "importance_row",
+    "MODE_ANCHOR", "state_errors", "AnchorState", "anchor_plan", "anchor_update",
 ]
 
 
@@ -488,6 +505,115 @@ def state_importance(cache: StateCache, L: Dict[Tuple[int, int], float], S: int,
                         tot += math.exp(lk - lt)
             w[t, k] = tot / (len(heads) * (q1 - q0))
     return w
+
+
+def state_errors(before: Dict[Tuple[int, int, int], Tuple[np.ndarray, float]], fresh, S: int, P: int,
+                 nseg: int) -> Tuple[np.ndarray, np.ndarray]:
+    """[DT] state error of the key sets computed in a step: for every
+    (query tile, key set) the sums over the tile's rows, the heads and the D
+    columns of (OUT_fresh - OUT_cached)^2 and of OUT_fresh^2, where
+    ``before`` is the cache's slot dictionary (k, h, row) -> (OUT, LSE) taken
+    before the step and ``fresh`` the dict partition_step returns.  Pairs not
+    computed, or whose slot held no state, are NaN.  The relative error is
+    sqrt(diff / norm).  Returns float64 [nqt][nseg] (diff, norm)."""
+    tiles = query_tiles(S, P)
+    starts = np.array([t[1] for t in tiles])
+    diff = np.full((len(tiles), nseg), np.nan)
+    norm = np.full((len(tiles), nseg), np.nan)
+    for (k, h), items in fresh.items():
+        for rs, (o_f, _l_f) in items:
+            t = int(np.searchsorted(starts, rs[0], side="right") - 1)
+            if any((k, h, int(r)) not in before for r in rs):
+                continue
+            o_c = np.stack([before[(k, h, int(r))][0] for r in rs])
+            if np.isnan(diff[t, k]):
+                diff[t, k] = norm[t, k] = 0.0
+            diff[t, k] += float(np.sum((o_f - o_c) ** 2))
+            norm[t, k] += float(np.sum(o_f ** 2))
+    return diff, norm
+
+
+class AnchorState:
+    """Host state of the anchor-guided planner: importance w and scale ratio
+    alpha per (query tile, key set), the local drift accumulated since the
+    last anchor per query tile, the threshold epsilon, the drift budget theta
+    and the target reuse ratio rho."""
+
+    def __init__(self, nqt: int, nseg: int, rho: float, theta: float):
+        self.w = np.zeros((nqt, nseg), dtype=np.float32)
+        self.alpha = np.ones((nqt, nseg), dtype=np.float32)
+        self.drift = np.zeros(nqt, dtype=np.float32)
+        self.eps = np.float32(0.0)
+        self.rho = float(rho)
+        self.theta = np.float32(theta)
+        self.last_anchor = 0
+
+
+def _local_set(S: int, P: int, group: int, t: int) -> int:
+    return 0 if group else query_tiles(S, P)[t][0]
+
+
+def anchor_plan(st: AnchorState, stamps: np.ndarray, step: int, S: int, P: int, group: int = 0):
+    """[DT] selection strategy with anchor steps.  Returns (plan, anchored).
+    An anchor (every set computed) is taken at step 1 or when any tile's
+    accumulated local drift exceeds theta; otherwise set k of tile t is
+    reused iff it is not the local set, its slot holds a state and
+    w * alpha * (step - t_c) <= epsilon, the products in float32."""
+    nqt, nseg = stamps.shape
+    anchored = step <= 1 or bool(np.any(st.drift > st.theta))
+    plan = np.full((nqt, nseg), COMPUTE, dtype=np.uint8)
+    if anchored:
+        return plan, True
+    for t in range(nqt):
+        loc = _local_set(S, P, group, t)
+        for k in range(nseg):
+            if k == loc or stamps[t, k] < 0:
+                continue
+            ase = np.float32(st.w[t, k]) * np.float32(st.alpha[t, k]) * np.float32(step - int(stamps[t, k]))
+            if ase <= st.eps:
+                plan[t, k] = REUSE
+    return plan, False
+
+
+def anchor_update(st: AnchorState, step: int, anchored: bool, stamps_before: np.ndarray, diff: np.ndarray,
+                  norm: np.ndarray, S: int, P: int, group: int = 0, w_now: Optional[np.ndarray] = None) -> None:
+    """[DT] metadata after a step: the local drift of every tile (its own
+    set's state error) accumulates since the last anchor; at an anchor the
+    importance is replaced by ``w_now``, every other set with a previous
+    state gets alpha = e / (step - t_c), the drift restarts at zero, and
+    epsilon becomes the rho-quantile of w * alpha over all (tile, non-local
+    set) pairs: the ceil(rho N)-th smallest value (0 if that count is 0).
+    Errors come in as (diff, norm) sums; e = sqrt(diff / norm), 0 when
+    norm is 0."""
+    nqt, nseg = stamps_before.shape
+
+    def err(t, k):
+        if np.isnan(diff[t, k]):
+            return None
+        return float(np.float32(math.sqrt(diff[t, k] / norm[t, k]))) if norm[t, k] > 0 else 0.0
+
+    if anchored:
+        st.drift[:] = 0.0
+        st.last_anchor = step
+        if w_now is not None:
+            st.w[:] = np.asarray(w_now, dtype=np.float32)
+        for t in range(nqt):
+            loc = _local_set(S, P, group, t)
+            for k in range(nseg):
+                if k == loc or stamps_before[t, k] < 0:
+                    continue
+                e = err(t, k)
+                if e is not None:
+                    st.alpha[t, k] = np.float32(e) / np.float32(step - int(stamps_before[t, k]))
+        rates = sorted(float(np.float32(st.w[t, k]) * np.float32(st.alpha[t, k]))
+                       for t in range(nqt) for k in range(nseg) if k != _local_set(S, P, group, t))
+        n = int(math.ceil(st.rho * len(rates) - 1e-9)) if rates else 0
+        st.eps = np.float32(rates[n - 1]) if n > 0 else np.float32(0.0)
+    else:
+        for t in range(nqt):
+            e = err(t, _local_set(S, P, group, t))
+            if e is not None:
+                st.drift[t] = np.float32(st.drift[t] + np.float32(e))
 
 
 def _get_or_identity(cache: StateCache, k, h, rs, D):
