@@ -78,6 +78,9 @@ extern "C" {
 #define DT_MODE_IMPORTANCE  5  /* step 1: anchor; later steps: the r key sets of smallest
                                   predicted error (importance x cache age) are reused;
                                   built by dt_plan_build_importance */
+#define DT_MODE_ANCHOR      6  /* anchor-guided: anchors triggered by local drift, reuse
+                                  by a threshold adapted at anchors; built by
+                                  dt_plan_build_anchor (below) */
 
 #define DT_PLAN_REUSE   0
 #define DT_PLAN_COMPUTE 1
@@ -169,6 +172,58 @@ DT_API int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, 
  * and counts as dt_plan_build.  Host only.  Errors: DT_ERR_INVALID. */
 DT_API int dt_plan_build_importance(const dt_plan_params* p, const float* weights, dt_plan* out);
 
+/* ---- anchor-guided planning ("DiTango", selection strategy and anchor
+ * steps; the equations are lost, these are the readings the prose supports).
+ * The state error of a key set computed at step t is ||OUT_t - OUT_c|| /
+ * ||OUT_t|| (Frobenius over the query tile's rows, all heads and D), OUT_c
+ * being the OUT its cache slot held; a tile's local drift is that error of
+ * its own key set (partition q, or set 0 with grouping), which every step
+ * computes.  An anchor (every set computed) is taken at step 1 and when the
+ * drift accumulated since the last anchor exceeds theta for any tile.  At an
+ * anchor the scale ratio of every other set with a previous state becomes
+ * alpha = e / (t - t_c) (error per step of cache age), and epsilon becomes
+ * the target_ratio-quantile of w * alpha over all (tile, non-local set)
+ * pairs (the ceil(target_ratio * N)-th smallest, 0 if that count is 0).
+ * Between anchors set k of a tile is reused iff it is not the local set, its
+ * slot holds a state and w * alpha * (t - t_c) <= epsilon (float32 products
+ * in that order). */
+typedef struct {
+  float* weights;             /* host [nqt][nseg]: importance w, replaced at anchors (in/out) */
+  float* alpha;               /* host [nqt][nseg]: scale ratios, 1 until measured (in/out) */
+  float* drift;               /* host [nqt]: local drift accumulated since the last anchor (in/out) */
+  float eps;                  /* reuse threshold epsilon (in/out) */
+  float theta;                /* drift budget that triggers an anchor (in) */
+  float target_ratio;         /* share of (tile, non-local set) pairs reused right after an anchor (in) */
+  int32_t last_anchor;        /* step of the last anchor, 0 = none (in/out) */
+  int32_t anchored;           /* (out) 1 if the plan dt_plan_build_anchor built last is an anchor */
+} dt_anchor_state;
+
+/* Initial planner state: w = 0, alpha = 1, drift = 0, eps = 0, last_anchor =
+ * 0, anchored = 0 (theta and target_ratio are the caller's).  The three
+ * arrays are caller-allocated host memory sized by dt_plan_geometry.  Host
+ * only.  Errors: DT_ERR_INVALID. */
+DT_API int dt_anchor_init(const dt_plan_params* p, dt_anchor_state* a);
+
+/* Plan of one step in DT_MODE_ANCHOR (p->mode must be DT_MODE_ANCHOR; either
+ * key-set layout): an anchor or the threshold rule above; sets a->anchored;
+ * then stamps and counts as dt_plan_build.  Host only.  Errors:
+ * DT_ERR_INVALID. */
+DT_API int dt_plan_build_anchor(const dt_plan_params* p, dt_anchor_state* a, dt_plan* out);
+
+/* Planner metadata after a step ran through dt_attn_partial_fused_tracked
+ * with the plan of dt_plan_build_anchor.  stamps_before: host [nqt][nseg],
+ * the stamps before that plan was built; plan: that plan; err: host copy of
+ * the step's d_err (layout below); weights_now: host [nqt][nseg] importance
+ * measured after the step (dt_state_importance), used and required only
+ * when a->anchored.  The error of a pair is sqrt(sum diff / sum norm) over
+ * its heads and warps in increasing order (double sums), rounded to float;
+ * pairs whose stamp was < 0 have no previous state and are skipped.  At an
+ * anchor: drift = 0, last_anchor = step, w = weights_now, alpha and epsilon
+ * as above; otherwise each tile's drift += its local error.  Host only.
+ * Errors: DT_ERR_INVALID. */
+DT_API int dt_anchor_update(const dt_plan_params* p, dt_anchor_state* a, const int32_t* stamps_before,
+                     const uint8_t* plan, const float* err, const float* weights_now);
+
 /* Fused step on the GPU ("DiTango", attention state Eq. 1-3, composition Eq. 4,
  * selective reuse Fig. 6).  For each head and query tile and each key set of
  * the tile's plan row (a partition, a group of partitions with p->group >= 1,
@@ -214,6 +269,22 @@ DT_API int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head_beg
                           const uint8_t* d_plan, const void* Q, const void* K, const void* V,
                           float* cache_O, float* cache_L, float* R, void* O, float* L,
                           int64_t* d_counters, int32_t* d_status, void* stream);
+
+/* The fused step of dt_attn_partial_fused that also measures state errors
+ * for the anchor-guided planner: for every (query tile, key set) it computes
+ * (all of them if err_all, else only the tile's local set) it reads the
+ * slot's previous OUT before overwriting it and writes, per head and per
+ * group of 32 rows (4 per tile), the sums over those rows and the D columns
+ * of (OUT_new - OUT_old)^2 and OUT_new^2 to
+ *   d_err fp32 [nqt][nseg][H][4][2]  (device; entries of pairs not measured
+ *                                     are left as they were).
+ * Partition modes only (fp32 or bf16 states).  Errors: those of
+ * dt_attn_partial_fused; DT_ERR_INVALID for window mode or a null d_err. */
+DT_API int dt_attn_partial_fused_tracked(const dt_plan_params* p, const uint8_t* d_plan,
+                          const void* Q, const void* K, const void* V,
+                          float* cache_O, float* cache_L, void* O, float* L,
+                          int64_t* d_counters, int32_t* d_status,
+                          float* d_err, int32_t err_all, void* stream);
 
 /* N-way composition of states ("DiTango", composition of attention states,
  * Eq. 4): for every row, L = M + ln sum_n e^(L_n - M), M = max_n L_n,

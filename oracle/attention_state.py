@@ -544,7 +544,7 @@ class AnchorState:
         self.alpha = np.ones((nqt, nseg), dtype=np.float32)
         self.drift = np.zeros(nqt, dtype=np.float32)
         self.eps = np.float32(0.0)
-        self.rho = float(rho)
+        self.rho = float(np.float32(rho))      # a float32 parameter, like the library's
         self.theta = np.float32(theta)
         self.last_anchor = 0
 

@@ -27,10 +27,13 @@ __all__ = [
     "DT_WR_APPLY", "DT_TILE", "DT_STATE_F32", "DT_STATE_BF16", "DT_MODE_IMPORTANCE",
     "dt_plan_build_importance", "dt_state_importance", "dt_share_output", "dt_key_set_tiles",
     "dt_attn_cfg_shared", "dt_plan_share_counts", "DT_SHARE_CFG", "DT_SHARE_TIMESTEP",
+    "DT_MODE_ANCHOR", "AnchorState", "dt_anchor_init", "dt_plan_build_anchor", "dt_anchor_update",
+    "dt_attn_partial_fused_tracked",
 ]
 
 DT_OK, DT_ERR_INVALID, DT_ERR_UNSUPPORTED, DT_ERR_CACHE_EMPTY, DT_ERR_CUDA, DT_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 DT_MODE_IMPORTANCE = 5
+DT_MODE_ANCHOR = 6
 DT_STATE_F32, DT_STATE_BF16 = 0, 1
 DT_MODE_ALL_COMPUTE, DT_MODE_PROXIMITY, DT_MODE_ALL_REUSE, DT_MODE_EXPLICIT, DT_MODE_WINDOW = 0, 1, 2, 3, 4
 DT_PLAN_REUSE, DT_PLAN_COMPUTE = 0, 1
@@ -55,6 +58,14 @@ class Plan(ctypes.Structure):
     _fields_ = [("plan", ctypes.POINTER(ctypes.c_uint8)), ("stamps", ctypes.POINTER(ctypes.c_int32)),
                 ("computed_blocks", ctypes.c_int64), ("skipped_blocks", ctypes.c_int64),
                 ("computed_flops", ctypes.c_int64), ("nqt", ctypes.c_int32), ("nseg", ctypes.c_int32)]
+
+
+class AnchorState(ctypes.Structure):
+    """dt_anchor_state: the host arrays are numpy buffers kept alive by the
+    Python object (see new_anchor_state)."""
+    _fields_ = [("weights", ctypes.POINTER(ctypes.c_float)), ("alpha", ctypes.POINTER(ctypes.c_float)),
+                ("drift", ctypes.POINTER(ctypes.c_float)), ("eps", ctypes.c_float), ("theta", ctypes.c_float),
+                ("target_ratio", ctypes.c_float), ("last_anchor", ctypes.c_int32), ("anchored", ctypes.c_int32)]
 
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -90,6 +101,10 @@ def load() -> ctypes.CDLL:
             "dt_share_output": ([i32, i32, i32, vp, vp, vp, vp, vp], ctypes.c_int),
             "dt_attn_cfg_shared": ([pp] + [vp] * 12, ctypes.c_int),
             "dt_plan_share_counts": ([pp, i32, ctypes.POINTER(Plan)], ctypes.c_int),
+            "dt_anchor_init": ([pp, ctypes.POINTER(AnchorState)], ctypes.c_int),
+            "dt_plan_build_anchor": ([pp, ctypes.POINTER(AnchorState), ctypes.POINTER(Plan)], ctypes.c_int),
+            "dt_anchor_update": ([pp, ctypes.POINTER(AnchorState), vp, vp, vp, vp], ctypes.c_int),
+            "dt_attn_partial_fused_tracked": ([pp] + [vp] * 11 + [i32, vp], ctypes.c_int),
             "dt_key_set_tiles": ([pp, i32, i32, vp, vp, i32], ctypes.c_int),
             "dt_set_wait_limit_ns": ([i64], ctypes.c_int),
         }
@@ -215,6 +230,57 @@ def dt_plan_share_counts(p: PlanParams, kind: int, counts: Optional[dict] = None
     _check(load().dt_plan_share_counts(ctypes.byref(p), kind, ctypes.byref(io)), "dt_plan_share_counts")
     return {"computed_blocks": io.computed_blocks, "skipped_blocks": io.skipped_blocks,
             "computed_flops": io.computed_flops}
+
+
+def new_anchor_state(p: PlanParams, target_ratio: float, theta: float):
+    """A dt_anchor_state with its host arrays, initialised by dt_anchor_init.
+    Returns (state, arrays) where arrays = {"weights", "alpha", "drift"} are
+    the numpy views the state points into (keep them alive)."""
+    nqt, nseg = dt_plan_geometry(p)
+    arr = {"weights": np.zeros((max(nqt, 1), nseg), np.float32), "alpha": np.zeros((max(nqt, 1), nseg), np.float32),
+           "drift": np.zeros(max(nqt, 1), np.float32)}
+    fp = ctypes.POINTER(ctypes.c_float)
+    st = AnchorState(arr["weights"].ctypes.data_as(fp), arr["alpha"].ctypes.data_as(fp),
+                     arr["drift"].ctypes.data_as(fp), 0.0, theta, target_ratio, 0, 0)
+    dt_anchor_init(p, st)
+    return st, arr
+
+
+def dt_anchor_init(p: PlanParams, st: AnchorState) -> None:
+    _check(load().dt_anchor_init(ctypes.byref(p), ctypes.byref(st)), "dt_anchor_init")
+
+
+def dt_plan_build_anchor(p: PlanParams, st: AnchorState, stamps: Optional[np.ndarray] = None):
+    """Anchor-guided plan of one step (p.mode = DT_MODE_ANCHOR).  Returns
+    (plan, counts, anchored); ``stamps`` is updated in place when given."""
+    nqt, nseg = dt_plan_geometry(p)
+    plan = np.zeros((nqt, nseg), dtype=np.uint8)
+    out = Plan()
+    out.plan = plan.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+    if stamps is not None:
+        assert stamps.dtype == np.int32 and stamps.flags.c_contiguous and stamps.size == nqt * nseg
+        out.stamps = stamps.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    _check(load().dt_plan_build_anchor(ctypes.byref(p), ctypes.byref(st), ctypes.byref(out)), "dt_plan_build_anchor")
+    return plan, {"computed_blocks": out.computed_blocks, "skipped_blocks": out.skipped_blocks,
+                  "computed_flops": out.computed_flops}, bool(st.anchored)
+
+
+def dt_anchor_update(p: PlanParams, st: AnchorState, stamps_before: np.ndarray, plan: np.ndarray, err: np.ndarray,
+                     weights_now: Optional[np.ndarray] = None) -> None:
+    sb = np.ascontiguousarray(stamps_before, dtype=np.int32)
+    pl = np.ascontiguousarray(plan, dtype=np.uint8)
+    e = np.ascontiguousarray(err, dtype=np.float32)
+    w = None if weights_now is None else np.ascontiguousarray(weights_now, dtype=np.float32)
+    _check(load().dt_anchor_update(ctypes.byref(p), ctypes.byref(st), _ptr(sb), _ptr(pl), _ptr(e), _ptr(w)),
+           "dt_anchor_update")
+
+
+def dt_attn_partial_fused_tracked(p: PlanParams, d_plan, Q, K, V, cache_O, cache_L, O, L, d_counters, d_status,
+                                  d_err, err_all: bool, stream=None) -> None:
+    _check(load().dt_attn_partial_fused_tracked(ctypes.byref(p), _ptr(d_plan), _ptr(Q), _ptr(K), _ptr(V),
+                                                _ptr(cache_O), _ptr(cache_L), _ptr(O), _ptr(L), _ptr(d_counters),
+                                                _ptr(d_status), _ptr(d_err), 1 if err_all else 0, _stream(stream)),
+           "dt_attn_partial_fused_tracked")
 
 
 def dt_attn_partial_fused(p: PlanParams, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,

@@ -74,11 +74,34 @@ extern "C" int dt_set_wait_limit_ns(int64_t ns) {
   return DT_OK;
 }
 
+namespace {
+int fused_step(const dt_plan_params* p, int32_t head_begin, int32_t head_count, const uint8_t* d_plan, const void* Q,
+               const void* K, const void* V, float* cache_O, float* cache_L, float* R, void* O, float* L,
+               int64_t* d_counters, int32_t* d_status, float* d_err, int err_all, void* stream);
+}  // namespace
+
 extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head_begin, int32_t head_count,
                                            const uint8_t* d_plan, const void* Q, const void* K, const void* V,
                                            float* cache_O, float* cache_L, float* R, void* O, float* L,
                                            int64_t* d_counters, int32_t* d_status, void* stream) {
-  if (!p || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE) return DT_ERR_INVALID;
+  return fused_step(p, head_begin, head_count, d_plan, Q, K, V, cache_O, cache_L, R, O, L, d_counters, d_status,
+                    nullptr, 0, stream);
+}
+
+extern "C" int dt_attn_partial_fused_tracked(const dt_plan_params* p, const uint8_t* d_plan, const void* Q,
+                                             const void* K, const void* V, float* cache_O, float* cache_L, void* O,
+                                             float* L, int64_t* d_counters, int32_t* d_status, float* d_err,
+                                             int32_t err_all, void* stream) {
+  if (!p || p->mode == DT_MODE_WINDOW || !d_err) return DT_ERR_INVALID;
+  return fused_step(p, 0, p->H, d_plan, Q, K, V, cache_O, cache_L, nullptr, O, L, d_counters, d_status, d_err,
+                    err_all, stream);
+}
+
+namespace {
+int fused_step(const dt_plan_params* p, int32_t head_begin, int32_t head_count, const uint8_t* d_plan, const void* Q,
+               const void* K, const void* V, float* cache_O, float* cache_L, float* R, void* O, float* L,
+               int64_t* d_counters, int32_t* d_status, float* d_err, int err_all, void* stream) {
+  if (!p || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_ANCHOR) return DT_ERR_INVALID;
   const bool win = p->mode == DT_MODE_WINDOW;
   if (!shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (win ? p->window < 1 : p->P < 1) return DT_ERR_INVALID;
@@ -96,7 +119,7 @@ extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head
   for (const void* q : ptrs)
     if (!aligned16(q)) return DT_ERR_UNSUPPORTED;
   if ((cache_O && !aligned16(cache_O)) || (cache_L && !aligned16(cache_L)) || (R && !aligned16(R)) ||
-      (d_counters && !aligned16(d_counters)))
+      (d_counters && !aligned16(d_counters)) || (d_err && !aligned16(d_err)))
     return DT_ERR_UNSUPPORTED;
 
   dt::Geom G = dt::make_geom(p->H, p->S, p->D, win ? 1 : p->P, win ? p->window : 0, win ? 0 : p->group);
@@ -129,6 +152,8 @@ extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head
   kp.item_end = (head_begin + head_count) * G.nqt;
   kp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->D));
   kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
+  kp.err = d_err;
+  kp.err_all = err_all ? 1 : 0;
   int sms = 0;
   if (int e = sm_count(&sms)) return e;
   const int n_items = kp.item_end - kp.item0;
@@ -136,6 +161,7 @@ extern "C" int dt_attn_partial_fused_heads(const dt_plan_params* p, int32_t head
   int grid = n_items < sms ? n_items : sms;
   return dt::launch_attn_fused(kp, dp, grid, reinterpret_cast<cudaStream_t>(stream));
 }
+}  // namespace
 
 extern "C" int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan, const void* Q, const void* K,
                                      const void* V, float* cache_O, float* cache_L, float* R, void* O, float* L,
@@ -161,7 +187,7 @@ extern "C" int dt_state_merge(int32_t N, int32_t H, int32_t S, int32_t D, const 
 extern "C" int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_plan, const float* fresh_O,
                                      const float* fresh_L, float* cache_O, float* cache_L, int32_t* d_status,
                                      void* stream) {
-  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE)
+  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_ANCHOR)
     return DT_ERR_INVALID;
   if (p->P < 1 || p->group < 0 || p->D < 4 || p->D % 4 != 0 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   if (p->state_dtype != DT_STATE_F32) return DT_ERR_UNSUPPORTED;
@@ -179,7 +205,7 @@ extern "C" int dt_state_cache_update(const dt_plan_params* p, const uint8_t* d_p
 
 extern "C" int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t* stamps, float* cache_O,
                                 float* cache_L, int32_t* d_status, void* stream) {
-  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE)
+  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_ANCHOR)
     return DT_ERR_INVALID;
   if (p->P < 1 || p->group < 1 || factor < 2 || factor > 8) return DT_ERR_INVALID;
   if (p->state_dtype != DT_STATE_F32) return DT_ERR_UNSUPPORTED;
@@ -218,7 +244,7 @@ extern "C" int dt_group_compose(const dt_plan_params* p, int32_t factor, int32_t
 
 extern "C" int dt_state_importance(const dt_plan_params* p, const float* cache_L, const float* L, float* d_weights,
                                    int32_t* d_status, void* stream) {
-  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE)
+  if (!p || p->mode == DT_MODE_WINDOW || p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_ANCHOR)
     return DT_ERR_INVALID;
   if (p->P < 1 || p->group < 0 || p->D < 1 || !shape_ok(p->H, p->S, p->D)) return DT_ERR_INVALID;
   const dt::Geom G = dt::make_geom(p->H, p->S, p->D, p->P, 0, p->group);

@@ -25,6 +25,8 @@ struct AttnParams {
   int item0, item_end;              // items [item0, item_end) of the H * nqt (head-major) items
   int state_bf16;                   // cached OUT is bf16 (cache_O then points to bf16 data)
   float scale_log2;                 // log2(e) / sqrt(D)
+  float* err;                       // state errors [nqt][nseg][H][4][2] (tracked step) or null
+  int err_all;                      // measure every computed key set (else only the local one)
   uint64_t wait_limit_ns;
 };
 

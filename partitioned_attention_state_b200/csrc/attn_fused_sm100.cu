@@ -821,6 +821,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const bool make_r = WIN && seg == 1;
         const float inv_tot = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
         const float inv_new = l_new > 0.f ? 1.f / l_new : 0.f;
+        // state error of this key set (anchor-guided planning): the slot's
+        // previous OUT is read before it is overwritten
+        const bool track = !WIN && p.err != nullptr &&
+                           (p.err_all || seg == (KM == kModeGrouped ? 0 : query_tile<KM>(G, qt).part));
+        float e_diff = 0.f, e_norm = 0.f;
 #pragma unroll
         for (int c = 0; c < D; c += 4) {
           float old[4], nw[4], x[4];
@@ -833,6 +838,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             nw[k] = fmaf(a, old[k], b * x[k]);
           }
           *oc = make_float4(nw[0], nw[1], nw[2], nw[3]);
+          if (valid && track) {
+            float ov[4];
+            if (CBF) {
+              const uint2 hv = __ldcs(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.cache_O) + slot * D + c));
+              ov[0] = bf16lo(hv.x); ov[1] = bf16hi(hv.x); ov[2] = bf16lo(hv.y); ov[3] = bf16hi(hv.y);
+            } else {
+              const float4 v4 = __ldcs(reinterpret_cast<const float4*>(p.cache_O + slot * D + c));
+              ov[0] = v4.x; ov[1] = v4.y; ov[2] = v4.z; ov[3] = v4.w;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float nv = x[k] * inv_l;
+              e_diff = fmaf(nv - ov[k], nv - ov[k], e_diff);
+              e_norm = fmaf(nv, nv, e_norm);
+            }
+          }
           if (valid) {
             if (!WIN && CBF) {
               uint2 pk;
@@ -850,6 +871,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
               v.w = nw[3] * inv_new - old[3] * inv_tot;
               __stcs(reinterpret_cast<float4*>(p.R + ((size_t)h * G.S + qrow) * D + c), v);
             }
+          }
+        }
+        if (track) {
+          // sums over the warp's 32 rows, then one entry per (tile, set, head, warp)
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            e_diff += __shfl_xor_sync(0xffffffffu, e_diff, o);
+            e_norm += __shfl_xor_sync(0xffffffffu, e_norm, o);
+          }
+          if (lane == 0) {
+            float* e2 = p.err + ((((size_t)qt * G.P + seg) * G.H + h) * 4 + q4) * 2;
+            e2[0] = e_diff;
+            e2[1] = e_norm;
           }
         }
         if (!WIN && valid) __stcs(p.cache_L + slot, nonempty ? (m_s + lg2(l_s)) * kLn2 : kNegInf);

@@ -9,6 +9,8 @@
 // expressed as two key sets per query tile (window, complement).  State
 // grouping (grouping of spatially adjacent states) makes a key set a group of
 // partitions; the proximity rule then ranks groups.
+#include <algorithm>
+#include <cmath>
 #include <cstring>
 #include <vector>
 
@@ -20,7 +22,7 @@ namespace {
 bool params_ok(const dt_plan_params* p) {
   if (!p) return false;
   if (p->H < 0 || p->S < 0 || p->D < 1 || p->step < 1) return false;
-  if (p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_IMPORTANCE) return false;
+  if (p->mode < DT_MODE_ALL_COMPUTE || p->mode > DT_MODE_ANCHOR) return false;
   if (p->group < 0) return false;
   if (p->mode == DT_MODE_WINDOW) {
     if (p->window < 1 || p->group != 0) return false;
@@ -128,7 +130,7 @@ int finish_plan(const dt_plan_params* p, const dt::Geom& g, dt_plan* out);
 
 extern "C" int dt_plan_build(const dt_plan_params* p, const uint8_t* explicit_plan, dt_plan* out) {
   if (!params_ok(p) || !out || !out->plan) return DT_ERR_INVALID;
-  if (p->mode == DT_MODE_IMPORTANCE) return DT_ERR_INVALID;       // needs weights
+  if (p->mode == DT_MODE_IMPORTANCE || p->mode == DT_MODE_ANCHOR) return DT_ERR_INVALID;   // needs their state
   dt::Geom g = geom_of(p);
   const int nqt = g.nqt, nseg = g.P;
   out->nqt = nqt;
@@ -219,6 +221,103 @@ extern "C" int dt_plan_share_counts(const dt_plan_params* p, int32_t kind, dt_pl
   io->computed_blocks = 0;
   io->skipped_blocks = total;
   io->computed_flops = 0;
+  return DT_OK;
+}
+
+namespace {
+
+// The local key set of query tile qt: its own partition, or set 0 with grouping.
+int local_set(const dt::Geom& g, int qt) { return g.grp > 0 ? 0 : dt::query_tile<0>(g, qt).part; }
+
+bool anchor_state_ok(const dt_plan_params* p, const dt_anchor_state* a) {
+  return params_ok(p) && a && p->mode == DT_MODE_ANCHOR && a->weights && a->alpha && a->drift;
+}
+
+}  // namespace
+
+extern "C" int dt_anchor_init(const dt_plan_params* p, dt_anchor_state* a) {
+  if (!anchor_state_ok(p, a)) return DT_ERR_INVALID;
+  const dt::Geom g = geom_of(p);
+  const size_t n = (size_t)g.nqt * g.P;
+  for (size_t i = 0; i < n; ++i) { a->weights[i] = 0.f; a->alpha[i] = 1.f; }
+  for (int t = 0; t < g.nqt; ++t) a->drift[t] = 0.f;
+  a->eps = 0.f;
+  a->last_anchor = 0;
+  a->anchored = 0;
+  return DT_OK;
+}
+
+extern "C" int dt_plan_build_anchor(const dt_plan_params* p, dt_anchor_state* a, dt_plan* out) {
+  if (!anchor_state_ok(p, a) || !out || !out->plan) return DT_ERR_INVALID;
+  const dt::Geom g = geom_of(p);
+  const int nqt = g.nqt, nseg = g.P;
+  out->nqt = nqt;
+  out->nseg = nseg;
+  out->computed_blocks = out->skipped_blocks = out->computed_flops = 0;
+  bool anchor = p->step <= 1;
+  for (int t = 0; t < nqt && !anchor; ++t) anchor = a->drift[t] > a->theta;
+  a->anchored = anchor ? 1 : 0;
+  for (int qt = 0; qt < nqt; ++qt) {
+    uint8_t* row = out->plan + (size_t)qt * nseg;
+    for (int k = 0; k < nseg; ++k) row[k] = DT_PLAN_COMPUTE;
+    if (anchor) continue;
+    const int loc = local_set(g, qt);
+    const int32_t* st = out->stamps ? out->stamps + (size_t)qt * nseg : nullptr;
+    for (int k = 0; k < nseg; ++k) {
+      if (k == loc || !st || st[k] < 0) continue;
+      const float ase = (a->weights[(size_t)qt * nseg + k] * a->alpha[(size_t)qt * nseg + k]) * (float)(p->step - st[k]);
+      if (ase <= a->eps) row[k] = DT_PLAN_REUSE;
+    }
+  }
+  return finish_plan(p, g, out);
+}
+
+extern "C" int dt_anchor_update(const dt_plan_params* p, dt_anchor_state* a, const int32_t* stamps_before,
+                                const uint8_t* plan, const float* err, const float* weights_now) {
+  if (!anchor_state_ok(p, a) || !stamps_before || !plan || !err) return DT_ERR_INVALID;
+  if (a->anchored && !weights_now) return DT_ERR_INVALID;
+  const dt::Geom g = geom_of(p);
+  const int nqt = g.nqt, nseg = g.P, H = p->H;
+  // error of pair (qt, k): sums over heads and the 4 row groups in increasing
+  // order, in double; false if the pair has no previous state or was not computed
+  auto pair_error = [&](int qt, int k, float* e) -> bool {
+    const size_t i = (size_t)qt * nseg + k;
+    if (plan[i] != DT_PLAN_COMPUTE || stamps_before[i] < 0) return false;
+    double diff = 0.0, norm = 0.0;
+    for (int h = 0; h < H; ++h)
+      for (int w = 0; w < 4; ++w) {
+        const float* e2 = err + (((i * H) + h) * 4 + w) * 2;
+        diff += (double)e2[0];
+        norm += (double)e2[1];
+      }
+    *e = norm > 0.0 ? (float)std::sqrt(diff / norm) : 0.f;
+    return true;
+  };
+  if (!a->anchored) {
+    for (int qt = 0; qt < nqt; ++qt) {
+      float e;
+      if (pair_error(qt, local_set(g, qt), &e)) a->drift[qt] = a->drift[qt] + e;
+    }
+    return DT_OK;
+  }
+  a->last_anchor = p->step;
+  std::vector<float> rates;
+  rates.reserve((size_t)nqt * nseg);
+  for (int qt = 0; qt < nqt; ++qt) {
+    a->drift[qt] = 0.f;
+    const int loc = local_set(g, qt);
+    for (int k = 0; k < nseg; ++k) {
+      const size_t i = (size_t)qt * nseg + k;
+      a->weights[i] = weights_now[i];
+      if (k == loc) continue;
+      float e;
+      if (pair_error(qt, k, &e)) a->alpha[i] = e / (float)(p->step - stamps_before[i]);
+      rates.push_back(a->weights[i] * a->alpha[i]);
+    }
+  }
+  std::sort(rates.begin(), rates.end());
+  const int64_t n = rates.empty() ? 0 : (int64_t)std::ceil((double)a->target_ratio * (double)rates.size() - 1e-9);
+  a->eps = n > 0 ? rates[(size_t)std::min<int64_t>(n, (int64_t)rates.size()) - 1] : 0.f;
   return DT_OK;
 }
 

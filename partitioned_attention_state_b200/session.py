@@ -20,10 +20,11 @@ from typing import Optional
 import numpy as np
 import torch
 
-from . import (DT_MODE_IMPORTANCE, DT_MODE_PROXIMITY, DT_MODE_WINDOW, DT_SHARE_CFG, DT_SHARE_TIMESTEP,
-               dt_attn_cfg_shared, dt_attn_partial_fused, dt_attn_partial_fused_heads, dt_group_compose,
-               dt_plan_build, dt_plan_build_importance, dt_plan_geometry, dt_plan_share_counts, dt_state_importance,
-               DtError, params)
+from . import (DT_MODE_ANCHOR, DT_MODE_IMPORTANCE, DT_MODE_PROXIMITY, DT_MODE_WINDOW, DT_SHARE_CFG,
+               DT_SHARE_TIMESTEP, dt_anchor_update, dt_attn_cfg_shared, dt_attn_partial_fused,
+               dt_attn_partial_fused_heads, dt_attn_partial_fused_tracked, dt_group_compose, dt_plan_build,
+               dt_plan_build_anchor, dt_plan_build_importance, dt_plan_geometry, dt_plan_share_counts,
+               dt_state_importance, new_anchor_state, DtError, params)
 
 
 def bf16_from_bits(bits: np.ndarray, device) -> torch.Tensor:
@@ -38,11 +39,15 @@ class Session:
 
     def __init__(self, H: int, S: int, D: int, P: int = 1, mode: int = DT_MODE_PROXIMITY, reuse_per_row: int = 0,
                  window: int = 0, device: str = "cuda", cache: bool = True, group: int = 0,
-                 state_dtype: int = 0):
+                 state_dtype: int = 0, target_ratio: float = 0.5, drift_budget: float = 0.5):
         """group: 0 = one key set (and cache slot) per partition; g >= 1 =
         state grouping (the local partition, then groups of g adjacent
         partitions); reuse_per_row then counts groups.  state_dtype:
-        DT_STATE_F32 or DT_STATE_BF16 (cached OUT in bf16, half the bytes)."""
+        DT_STATE_F32 or DT_STATE_BF16 (cached OUT in bf16, half the bytes).
+        mode DT_MODE_ANCHOR plans every step with the anchor-guided planner
+        (target_ratio: share of (tile, non-local set) pairs reused right after
+        an anchor; drift_budget: accumulated local drift that triggers an
+        anchor); its steps synchronise to read the measured state errors."""
         self.H, self.S, self.D, self.P = H, S, D, P
         self.mode, self.r, self.window = mode, reuse_per_row, window
         self.group = group
@@ -71,6 +76,13 @@ class Session:
         self.status = torch.zeros(4, dtype=torch.int32, device=dev)
         self.stamps = np.full((self.nqt, self.nseg), -1, dtype=np.int32)
         self.weights: Optional[np.ndarray] = None
+        self.anchor = None
+        if mode == DT_MODE_ANCHOR:
+            pa = params(H, S, D, P, DT_MODE_ANCHOR, 0, 0, 1, group, state_dtype)
+            self.anchor, self.anchor_arrays = new_anchor_state(pa, target_ratio, drift_budget)
+            self.d_err = torch.zeros((max(self.nqt, 1), self.nseg, H, 4, 2), dtype=torch.float32, device=dev)
+            self.last_err = None
+            self.last_anchored = False
         self.last_counts = None
         self.last_plan = None
 
@@ -142,11 +154,39 @@ class Session:
     def step(self, step: int, mode: Optional[int] = None, explicit: Optional[np.ndarray] = None,
              stream=None) -> dict:
         """Host plan build, asynchronous plan upload, one fused launch."""
+        if (self.mode if mode is None else mode) == DT_MODE_ANCHOR:
+            return self._step_anchor(step, stream)
         p, plan, counts = self.plan(step, mode, explicit)
         st = torch.cuda.current_stream(self.device) if stream is None else stream
         self._upload_plan(plan, st)
         self.launch(p, st)
         self._mark_plan_read(st)
+        self.last_counts, self.last_plan = counts, plan
+        return counts
+
+    def _step_anchor(self, step: int, stream=None) -> dict:
+        """One anchor-guided step: dt_plan_build_anchor, the tracked fused
+        launch (every computed set measured at an anchor, else the local
+        sets), then the state errors and, at an anchor, the importance read
+        back for dt_anchor_update.  Synchronises the stream."""
+        p = params(self.H, self.S, self.D, self.P, DT_MODE_ANCHOR, 0, 0, step, self.group, self.state_dtype)
+        before = self.stamps.copy()
+        plan, counts, anchored = dt_plan_build_anchor(p, self.anchor, self.stamps)
+        st = torch.cuda.current_stream(self.device) if stream is None else stream
+        self._upload_plan(plan, st)
+        dt_attn_partial_fused_tracked(p, self.d_plan, self.Q, self.K, self.V, self.cache_O, self.cache_L, self.O,
+                                      self.L, self.counters, self.status, self.d_err, anchored, st)
+        self._mark_plan_read(st)
+        w = None
+        if anchored:
+            d_w = torch.empty((max(self.nqt, 1), self.nseg), dtype=torch.float32, device=self.device)
+            dt_state_importance(p, self.cache_L, self.L, d_w, self.status, st)
+            w = d_w[: self.nqt].cpu().numpy()
+        st.synchronize()
+        self.check()
+        err = self.d_err[: self.nqt].cpu().numpy()
+        dt_anchor_update(p, self.anchor, before, plan, err, w)
+        self.last_err, self.last_anchored, self.weights = err, anchored, (w if anchored else self.weights)
         self.last_counts, self.last_plan = counts, plan
         return counts
 

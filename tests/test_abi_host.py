@@ -431,3 +431,85 @@ def test_share_calls_validated_on_the_host():
     assert lib.dt_attn_cfg_shared(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_INVALID
     p.H = 4
     assert lib.dt_attn_cfg_shared(ctypes.byref(p), *([None] * 11), None) == dt.DT_ERR_INVALID   # null buffers
+
+
+def _sum_errors(err, plan, stamps_before):
+    """(diff, norm) of the tracked pairs from the kernel's per-(head, warp)
+    partial sums, added in the library's order (heads, then row groups) in
+    float64; NaN where the pair has no previous state or was not computed."""
+    nqt, nseg, H = err.shape[:3]
+    diff = np.full((nqt, nseg), np.nan)
+    norm = np.full((nqt, nseg), np.nan)
+    for t in range(nqt):
+        for k in range(nseg):
+            if plan[t, k] != orc.COMPUTE or stamps_before[t, k] < 0:
+                continue
+            d = n = 0.0
+            for h in range(H):
+                for w in range(4):
+                    d += float(err[t, k, h, w, 0])
+                    n += float(err[t, k, h, w, 1])
+            diff[t, k], norm[t, k] = d, n
+    return diff, norm
+
+
+@pytest.mark.parametrize("S,P,g,rho", [(4096, 16, 0, 0.5), (4096, 16, 4, 0.4), (1800, 12, 0, 0.3), (2600, 7, 2, 0.75)])
+def test_anchor_planner_matches_oracle(S, P, g, rho):
+    """dt_plan_build_anchor / dt_anchor_update against the oracle's
+    anchor_plan / anchor_update on random measurements over 10 steps,
+    including drift-triggered anchors: plans, anchor decisions and every
+    piece of planner state bit-exact."""
+    H, D = 3, 64
+    p = dt.params(H, S, D, P, dt.DT_MODE_ANCHOR, 0, 0, 1, g)
+    nqt, nseg = dt.dt_plan_geometry(p)
+    theta = 0.05
+    st_c, arr = dt.new_anchor_state(p, rho, theta)
+    st_o = orc.AnchorState(nqt, nseg, rho, theta)
+    stamps_c = np.full((nqt, nseg), -1, np.int32)
+    stamps_o = stamps_c.copy()
+    rng = np.random.Generator(np.random.PCG64(S + P + g))
+    anchors = []
+    for step in range(1, 11):
+        p.step = step
+        before = stamps_c.copy()
+        plan_c, counts, anchored = dt.dt_plan_build_anchor(p, st_c, stamps_c)
+        plan_o, anch_o = orc.anchor_plan(st_o, stamps_o, step, S, P, g)
+        np.testing.assert_array_equal(plan_c, plan_o)
+        assert anchored == anch_o
+        anchors.append(anchored)
+        stamps_o[plan_o == orc.COMPUTE] = step
+        np.testing.assert_array_equal(stamps_c, stamps_o)
+        # measurements: small drifts, a large one at step 5
+        scale = 0.3 if step == 5 else 0.002
+        err = np.empty((nqt, nseg, H, 4, 2), np.float32)
+        err[..., 1] = rng.uniform(0.5, 2.0, (nqt, nseg, H, 4))
+        err[..., 0] = (err[..., 1] * rng.uniform(0.0, scale, (nqt, nseg, H, 4)) ** 2).astype(np.float32)
+        w_now = rng.uniform(0.0, 0.3, (nqt, nseg)).astype(np.float32) if anchored else None
+        dt.dt_anchor_update(p, st_c, before, plan_c, err, w_now)
+        diff, norm = _sum_errors(err, plan_c, before)
+        orc.anchor_update(st_o, step, anchored, before, diff, norm, S, P, g, w_now=w_now)
+        np.testing.assert_array_equal(arr["alpha"][:nqt], st_o.alpha)
+        np.testing.assert_array_equal(arr["drift"][:nqt], st_o.drift)
+        np.testing.assert_array_equal(arr["weights"][:nqt], st_o.w)
+        assert np.float32(st_c.eps) == st_o.eps
+    assert anchors[0] and anchors[5] and sum(anchors) >= 2      # the large drift of step 5 anchors step 6
+
+
+def test_anchor_calls_validated():
+    import ctypes
+    lib = dt.load()
+    p = dt.params(2, 1024, 64, 4, dt.DT_MODE_PROXIMITY, 1, 0, 1)
+    st = dt.AnchorState()
+    assert lib.dt_anchor_init(ctypes.byref(p), ctypes.byref(st)) == dt.DT_ERR_INVALID          # wrong mode, null arrays
+    p.mode = dt.DT_MODE_ANCHOR
+    assert lib.dt_anchor_init(ctypes.byref(p), ctypes.byref(st)) == dt.DT_ERR_INVALID          # null arrays
+    st2, _ = dt.new_anchor_state(p, 0.5, 0.1)
+    plan = dt.Plan()
+    assert lib.dt_plan_build_anchor(ctypes.byref(p), ctypes.byref(st2), ctypes.byref(plan)) == dt.DT_ERR_INVALID
+    st2.anchored = 1
+    z = np.zeros(64, np.int32)
+    assert lib.dt_anchor_update(ctypes.byref(p), ctypes.byref(st2), z.ctypes.data, z.ctypes.data, z.ctypes.data,
+                                None) == dt.DT_ERR_INVALID                                       # anchor needs weights
+    pw = dt.params(1, 1024, 64, 1, dt.DT_MODE_WINDOW, 0, 64, 1)
+    assert lib.dt_attn_partial_fused_tracked(ctypes.byref(pw), *([None] * 11), 0, None) == dt.DT_ERR_INVALID
+    assert lib.dt_plan_build(ctypes.byref(p), None, ctypes.byref(plan)) == dt.DT_ERR_INVALID      # needs its state

@@ -634,3 +634,84 @@ def test_share_previous_output():
     assert np.array_equal(sess.stamps, st)
     assert counts["computed_blocks"] == 0 and counts["computed_flops"] == 0
     assert counts["skipped_blocks"] == w.H * 8 * 8
+
+
+# ------------------------------------------------- anchor-guided planning
+
+def _sum_err(err, plan, before, anchored, S, P, g):
+    """State errors of the pairs a step measured (every computed pair with a
+    previous state at an anchor, else the local sets) from the kernel's
+    partial sums (heads, then row groups, float64, the library's order); NaN
+    where not measured.  Returns (diff, norm)."""
+    nqt, nseg, H = err.shape[:3]
+    diff = np.full((nqt, nseg), np.nan)
+    norm = np.full((nqt, nseg), np.nan)
+    tiles = orc.query_tiles(S, P)
+    for t in range(nqt):
+        local = 0 if g else tiles[t][0]
+        for k in range(nseg):
+            if plan[t, k] != orc.COMPUTE or before[t, k] < 0 or not (anchored or k == local):
+                continue
+            d = n = 0.0
+            for h in range(H):
+                for w in range(4):
+                    d += float(err[t, k, h, w, 0])
+                    n += float(err[t, k, h, w, 1])
+            diff[t, k], norm[t, k] = d, n
+    return diff, norm
+
+
+@pytest.mark.parametrize("g,sd", [(0, 0), (2, 0), (0, 1)])
+def test_anchor_guided_schedule_matches_oracle(g, sd):
+    """DT_MODE_ANCHOR on the GPU: per step the plan and the anchor decision
+    equal the oracle planner's fed with the same measurements (bit-exact);
+    outputs and fresh states match the oracle run with that plan; the
+    measured state errors match the oracle's own; unchanged inputs measure
+    exactly zero drift; a large perturbation triggers an anchor at the next
+    step and small ones do not."""
+    H, S, D, P = 2, 2048, 64, 8
+    sess = Session(H, S, D, P, mode=dt.DT_MODE_ANCHOR, group=g, state_dtype=sd, target_ratio=0.5,
+                   drift_budget=0.5)
+    nqt, nseg = sess.nqt, sess.nseg
+    st_o = orc.AnchorState(nqt, nseg, 0.5, 0.5)
+    stamps_o = np.full((nqt, nseg), -1, np.int32)
+    cache = orc.StateCache(bf16=sd == dt.DT_STATE_BF16)
+    rng = np.random.Generator(np.random.PCG64(40 + g + sd))
+    master = [rng.standard_normal((H, S, D)).astype(np.float32) / np.float32(8.0) for _ in range(3)]
+    sigmas = [0.0, 0.0, 0.004, 0.004, 1.0, 0.004, 0.004]
+    anchors, reused = [], []
+    for step, sig in enumerate(sigmas, start=1):
+        for m in master:
+            m += np.float32(sig) * rng.standard_normal(m.shape).astype(np.float32)
+        q, k, v = (wl.f32_to_bf16_bits(m) for m in master)
+        sess.set_inputs(q, k, v)
+        before = sess.stamps.copy()
+        sess.step(step)
+        plan = sess.last_plan
+        plan_o, anch_o = orc.anchor_plan(st_o, stamps_o, step, S, P, g)
+        np.testing.assert_array_equal(plan, plan_o)
+        assert sess.last_anchored == anch_o
+        anchors.append(anch_o)
+        stamps_o[plan_o == orc.COMPUTE] = step
+        snap = dict(cache.slots)
+        O_ref, L_ref, fresh = orc.partition_step(q, k, v, plan, S, P, cache, group=g)
+        check_out(to_np(sess.O), O_ref, f"O step {step}")
+        check_lse(to_np(sess.L), L_ref, f"LSE step {step}")
+        # measured errors against the oracle's own
+        d_o, n_o = orc.state_errors(snap, fresh, S, P, nseg)
+        d_g, n_g = _sum_err(sess.last_err, plan, before, anch_o, S, P, g)
+        tracked = ~np.isnan(d_g)
+        assert tracked.any() or step == 1
+        e_g = np.sqrt(d_g[tracked] / n_g[tracked])
+        e_o = np.sqrt(d_o[tracked] / n_o[tracked])
+        np.testing.assert_allclose(e_g, e_o, rtol=0.05, atol=3e-3)
+        if sig == 0.0 and step > 1 and sd == dt.DT_STATE_F32:
+            assert np.all(d_g[tracked] == 0.0)          # identical inputs: the kernel reproduces its states exactly
+        # the oracle planner follows the same measurements
+        orc.anchor_update(st_o, step, anch_o, before, d_g, n_g, S, P, g,
+                          w_now=sess.weights if anch_o else None)
+        np.testing.assert_array_equal(sess.anchor_arrays["alpha"][:nqt], st_o.alpha)
+        np.testing.assert_array_equal(sess.anchor_arrays["drift"][:nqt], st_o.drift)
+        reused.append(int((plan == orc.REUSE).sum()))
+    assert anchors[0] and anchors[5] and not any(anchors[1:5])
+    assert reused[1] > 0 and reused[6] > 0              # steps after an anchor reuse states
