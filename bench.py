@@ -533,6 +533,39 @@ def main():
                    "GB/s": cbytes / (cms * 1e-3) / 1e9, "frac_of_hbm": cbytes / (cms * 1e-3) / 1e9 / hbm}
         del gs
 
+    # the anchor-guided planner on this workload: a short schedule with the
+    # workload's perturbation, each step planned by dt_plan_build_anchor,
+    # launched with state-error tracking and followed by dt_anchor_update
+    anchor_guided = None
+    if not win and grp == 0 and not args.no_grouped and args.heads is None:
+        asess = Session(w.H, w.S, w.D, w.P, mode=dt.DT_MODE_ANCHOR, target_ratio=0.5, drift_budget=0.25)
+        astream = wl.stream_for(w)
+        rows = []
+        for step in range(1, 7):
+            asess.set_inputs(*astream.next_step())
+            a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier()
+            t0 = time.perf_counter()
+            a_ev.record(cur)
+            c = asess.step(step)                 # synchronises: reads the measured errors back
+            b_ev.record(cur)
+            barrier()
+            wall = (time.perf_counter() - t0) * 1e3
+            rows.append({"step": step, "anchor": bool(asess.last_anchored), "ms": a_ev.elapsed_time(b_ev),
+                         "wall_ms": wall, "tflops": c["computed_flops"] / (a_ev.elapsed_time(b_ev) * 1e-3) / 1e12,
+                         "reuse_ratio": c["skipped_blocks"] / max(1, c["skipped_blocks"] + c["computed_blocks"]),
+                         "max_drift": float(asess.anchor_arrays["drift"][: asess.nqt].max()),
+                         "eps": float(asess.anchor.eps)})
+        asess.check()
+        non = [r for r in rows if not r["anchor"]]
+        anchor_guided = {"planner": "dt_plan_build_anchor (target_ratio 0.5, drift budget 0.25)",
+                         "steps": rows, "anchors": [r["step"] for r in rows if r["anchor"]],
+                         "mean_ms_non_anchor": float(np.mean([r["ms"] for r in non])) if non else None,
+                         "mean_reuse_ratio_non_anchor": float(np.mean([r["reuse_ratio"] for r in non])) if non else None,
+                         "timing": "CUDA events around each step (tracked launch, importance at anchors, error read-back)"}
+        del asess
+        torch.cuda.empty_cache()
+
     # every other workload of the hot-path table, timed like the headline
     # (anchor step, then graph replays of the reuse step), with the CPU
     # oracle on a bounded sample of each
@@ -648,6 +681,7 @@ def main():
             "group_compose": compose,
             "bf16_state_cache": bf16c,
             "importance": importance,
+            "anchor_guided": anchor_guided,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
