@@ -338,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           const QTile t = query_tile<KM>(G, qt);
           if (nq > 0 && !mbar_wait(&bars[C::bQEmpty], (nq - 1) & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim))
             goto tma_done;
+          DT_TR(19, nq);
           mbar_arrive_expect_tx(&bars[C::bQFull], C::kTileBytes);
           for (int c = 0; c < C::kN64; ++c)
             tma_load_3d_hint(sQ + c * C::kBlk, &p.tmQ, &bars[C::bQFull], 64 * c, t.q0, h, pol_once);
@@ -393,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const int rot = seg_rotation<WIN>(G, idx);
         if (!item_has_compute<KM>(G, qt, cm)) continue;
         if (!mbar_wait(&bars[C::bQFull], nq & 1, abort_flag, p.status, DT_ERR_TIMEOUT, lim)) { ok = false; break; }
+        DT_TR(20, nq);
         ++nq;
         tc_fence_after();
         for (int j = 0; j < G.P && ok; ++j) {
@@ -707,6 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           n_skip += counted_blocks<KM>(G, qt, seg);   // same in every lane; thread 0 reports
           ++n_read;
           if (WIN) { use_r = true; ++merged; continue; }   // complement reused: add R at the end
+          if (warp == kWarpEpi) DT_TR(17, n_read);
           const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
           const float lse_c = valid ? __ldcs(p.cache_L + slot) : kNegInf;
           const bool nonempty = lse_c > kNegInf;
@@ -763,6 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           have = have || nonempty;
           ++jr;
           ++merged;
+          if (warp == kWarpEpi) DT_TR(18, n_read);
           return;
         }
       };
@@ -915,6 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         }
         __stcs(p.L + (size_t)h * G.S + qrow, (have && l_tot > 0.f) ? (m_tot + lg2(l_tot)) * kLn2 : kNegInf);
       }
+      if (warp == kWarpEpi) DT_TR(16, (idx - p.item0) / gridDim.x);
     }
   ep_done:
     if (r == 0 && p.counters) {

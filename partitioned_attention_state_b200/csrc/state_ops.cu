@@ -168,21 +168,94 @@ __global__ void __launch_bounds__(kBlock) group_compose_kernel(int m, int factor
   }
 }
 
+// The same regrouping with every input of a row held at once (m <= MAXM old
+// groups, D <= 128 so that a lane owns one float4 of a row): all loads of the
+// row are issued before any store, so a row costs one memory round trip
+// instead of one per new group.  The warp synchronises once between its loads
+// and its stores, after which no old value of the row is read again.
+template <int MAXM>
+__global__ void __launch_bounds__(kBlock) group_compose_row_kernel(int m, int factor, int64_t rows, int D,
+                                                                   float* __restrict__ cO, float* __restrict__ cL) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (kBlock / 32);
+  const int m2 = (m + factor - 1) / factor;
+  const bool on = lane < D / 4;
+  for (int64_t row = blockIdx.x * (int64_t)(kBlock / 32) + (threadIdx.x >> 5); row < rows; row += warps) {
+    float lv[MAXM];
+    float4 v[MAXM];
+#pragma unroll
+    for (int k = 0; k < MAXM; ++k) {
+      lv[k] = k < m ? cL[(int64_t)(1 + k) * rows + row] : kNegInf;
+      v[k] = (k < m && on) ? __ldcs(reinterpret_cast<const float4*>(cO + ((int64_t)(1 + k) * rows + row) * D) + lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncwarp();
+    for (int i = 0; i < m2; ++i) {
+      const int j0 = factor * i, j1 = min(j0 + factor, m);
+      float M = kNegInf;
+#pragma unroll
+      for (int k = 0; k < MAXM; ++k)
+        if (k >= j0 && k < j1) M = fmaxf(M, lv[k]);
+      float Lr = kNegInf;
+      if (M > kNegInf) {
+        float tot = 0.f;
+#pragma unroll
+        for (int k = 0; k < MAXM; ++k)
+          if (k >= j0 && k < j1) tot += expf(lv[k] - M);
+        Lr = M + logf(tot);
+      }
+      // a slot with LSE -inf (possibly never written) gets weight 0 and is not read
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < MAXM; ++k) {
+        const float wk = (k >= j0 && k < j1 && lv[k] > kNegInf) ? expf(lv[k] - Lr) : 0.f;
+        if (wk != 0.f) {
+          acc.x = fmaf(wk, v[k].x, acc.x);
+          acc.y = fmaf(wk, v[k].y, acc.y);
+          acc.z = fmaf(wk, v[k].z, acc.z);
+          acc.w = fmaf(wk, v[k].w, acc.w);
+        }
+      }
+      if (on) __stcs(reinterpret_cast<float4*>(cO + ((int64_t)(1 + i) * rows + row) * D) + lane, acc);
+      if (lane == 0) cL[(int64_t)(1 + i) * rows + row] = Lr;
+    }
+  }
+}
+
 // "DiTango", partition importance: the normalised composition weight
 // exp(LSE_k - LSE) of key set k for each row, averaged over the rows of a
 // query tile and the heads.  One block per (query tile, key set).
-__global__ void __launch_bounds__(kBlock) state_importance_kernel(Geom G, const float* __restrict__ cL,
-                                                                  const float* __restrict__ L,
-                                                                  float* __restrict__ w) {
-  __shared__ float part[kBlock / 32];
+constexpr int kImpBlock = 128;   // one thread per row of a query tile
+__global__ void __launch_bounds__(kImpBlock) state_importance_kernel(Geom G, const float* __restrict__ cL,
+                                                                     const float* __restrict__ L,
+                                                                     float* __restrict__ w) {
+  __shared__ float part[kImpBlock / 32];
   const int qt = blockIdx.x / G.P, k = blockIdx.x - qt * G.P;
   const QTile t = query_tile<kModePartition>(G, qt);
   const int n = G.H * t.rows;
   float acc = 0.f;
-  for (int i = threadIdx.x; i < n; i += kBlock) {
-    const int h = i / t.rows, r = t.q0 + (i - h * t.rows);
-    const float lk = cL[((int64_t)k * G.H + h) * G.S + r], lt = L[(int64_t)h * G.S + r];
-    if (lk > kNegInf && lt > kNegInf) acc += expf(lk - lt);
+  if ((int)threadIdx.x < t.rows) {
+    // thread t owns row q0 + t and walks the heads with 8 loads of each array
+    // in flight; a warp's loads cover 32 consecutive rows (128 bytes)
+    const int r = t.q0 + threadIdx.x;
+    const float* lk = cL + (int64_t)k * G.H * G.S + r;
+    const float* lt = L + r;
+    int h = 0;
+    for (; h + 8 <= G.H; h += 8) {
+      float a[8], b[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        a[u] = __ldcs(lk + (int64_t)(h + u) * G.S);
+        b[u] = lt[(int64_t)(h + u) * G.S];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (a[u] > kNegInf && b[u] > kNegInf) acc += expf(a[u] - b[u]);
+    }
+    for (; h < G.H; ++h) {
+      const float a = __ldcs(lk + (int64_t)h * G.S), b = lt[(int64_t)h * G.S];
+      if (a > kNegInf && b > kNegInf) acc += expf(a - b);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -190,7 +263,7 @@ __global__ void __launch_bounds__(kBlock) state_importance_kernel(Geom G, const 
   __syncthreads();
   if (threadIdx.x == 0) {
     float tot = 0.f;
-    for (int j = 0; j < kBlock / 32; ++j) tot += part[j];
+    for (int j = 0; j < kImpBlock / 32; ++j) tot += part[j];
     w[blockIdx.x] = n > 0 ? tot / (float)n : 0.f;
   }
 }
@@ -271,6 +344,12 @@ int launch_cache_update(const Geom& G, const uint8_t* plan, const float* fO, con
 int launch_group_compose(int m, int factor, int H, int S, int D, float* cO, float* cL, int sms, cudaStream_t st) {
   const int64_t rows = (int64_t)H * S;
   const int grid = grid_for(rows * 32, sms);
+  if (D <= 128 && m <= 16) {   // every input of a row at once
+    if (m <= 4) group_compose_row_kernel<4><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL);
+    else if (m <= 8) group_compose_row_kernel<8><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL);
+    else group_compose_row_kernel<16><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL);
+    return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
+  }
   switch (factor) {   // the factor bounds how many inputs a lane loads at once
     case 2: group_compose_kernel<2><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL); break;
     case 3: group_compose_kernel<3><<<grid, kBlock, 0, st>>>(m, factor, rows, D, cO, cL); break;
@@ -282,7 +361,7 @@ int launch_group_compose(int m, int factor, int H, int S, int D, float* cO, floa
 
 int launch_state_importance(const Geom& G, const float* cL, const float* L, float* w, cudaStream_t st) {
   const int64_t blocks = (int64_t)G.nqt * G.P;
-  state_importance_kernel<<<(unsigned)blocks, kBlock, 0, st>>>(G, cL, L, w);
+  state_importance_kernel<<<(unsigned)blocks, kImpBlock, 0, st>>>(G, cL, L, w);
   return cudaGetLastError() == cudaSuccess ? DT_OK : DT_ERR_CUDA;
 }
 

@@ -445,7 +445,8 @@ def test_grouped_video_full_size_sampled_rows():
                            rows=sample_rows(w.S, w.P, n_extra=24), group=4)
 
 
-@pytest.mark.parametrize("P,g,f", [(8, 1, 2), (16, 2, 2), (12, 1, 3), (7, 2, 4), (12, 1, 5), (16, 1, 8)])
+# m = ceil(P / g) old groups: 4, 8 and 16 take the row-at-once kernel, 20 the group-by-group one
+@pytest.mark.parametrize("P,g,f", [(8, 1, 2), (16, 2, 2), (12, 1, 3), (7, 2, 4), (12, 1, 5), (16, 1, 8), (20, 1, 2)])
 def test_group_compose_matches_oracle(P, g, f):
     """Dynamic Group State Compose on the GPU: the regrouped cache equals the
     oracle's N-way composition of the GPU's own cached states (fp32 rounding
