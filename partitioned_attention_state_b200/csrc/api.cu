@@ -146,6 +146,7 @@ int fused_step(const dt_plan_params* p, int32_t head_begin, int32_t head_count, 
   kp.H = p->H; kp.S = p->S; kp.D = p->D; kp.P = win ? 1 : p->P; kp.window = win ? p->window : 0;
   kp.geom = G;
   kp.state_bf16 = p->state_dtype == DT_STATE_BF16;
+  kp.cache_v8 = (reinterpret_cast<uintptr_t>(cache_O) & 31u) == 0;
   // items are numbered over all heads, so a head range computes exactly what
   // the whole launch computes for those heads
   kp.item0 = head_begin * G.nqt;

@@ -24,6 +24,7 @@ struct AttnParams {
   Geom geom;                        // make_geom(H, S, D, P, window), read from the parameter bank
   int item0, item_end;              // items [item0, item_end) of the H * nqt (head-major) items
   int state_bf16;                   // cached OUT is bf16 (cache_O then points to bf16 data)
+  int cache_v8;                     // cache_O is 32-byte aligned (fp32 states stored 32 bytes at a time)
   float scale_log2;                 // log2(e) / sqrt(D)
   float* err;                       // state errors [nqt][nseg][H][4][2] (tracked step) or null
   int err_all;                      // measure every computed key set (else only the local one)

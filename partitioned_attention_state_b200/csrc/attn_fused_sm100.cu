@@ -711,7 +711,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           if (WIN) { use_r = true; ++merged; continue; }   // complement reused: add R at the end
           if (warp == kWarpEpi) DT_TR(17, n_read);
           const size_t slot = ((size_t)seg * G.H + h) * G.S + qrow;
+          // The warp's 32 slot rows are contiguous: lane l reads 16 bytes (8
+          // of bf16) of every row, so each load instruction covers one whole
+          // row.  All 32 rows and the rows' LSEs are loaded together (one
+          // memory round trip); rows past a ragged tile are not read, and
+          // rows whose state is empty (LSE -inf) are zeroed after the load.
+          const size_t row0 = slot - r + 32 * q4;           // slot row of the warp's first row
+          const bool lane_on = 4 * lane < D;
+          const uint32_t vrows = __ballot_sync(0xffffffffu, valid);
           const float lse_c = valid ? __ldcs(p.cache_L + slot) : kNegInf;
+          float4 cv[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const bool on = lane_on && ((vrows >> k) & 1u);
+            if (CBF) {
+              const uint2 hv = on ? __ldcs(reinterpret_cast<const uint2*>(
+                                        reinterpret_cast<const __nv_bfloat16*>(p.cache_O) + (row0 + k) * D) + lane)
+                                  : make_uint2(0, 0);
+              cv[k] = make_float4(bf16lo(hv.x), bf16hi(hv.x), bf16lo(hv.y), bf16hi(hv.y));
+            } else {
+              cv[k] = on ? __ldcs(reinterpret_cast<const float4*>(p.cache_O + (row0 + k) * D) + lane)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+          }
           const bool nonempty = lse_c > kNegInf;
           const float m_c = lse_c * kLog2e;
           float a, b, m_new;
@@ -722,43 +744,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             b = nonempty ? ex2(m_c - m_new) : 0.f;
           }
           const float l_new = a * l_tot + b;
-          // The warp's 32 slot rows are contiguous: lane l reads 16 bytes (8
-          // of bf16) of every row, so each load instruction covers one whole
-          // row; 16 rows are in flight together.  Rows the slot has no state
-          // for (ragged tile, empty state) are not read.
           const uint32_t live = __ballot_sync(0xffffffffu, valid && nonempty);
           __syncwarp();                                   // the lanes' own-row writes are visible
-          const size_t row0 = slot - r + 32 * q4;           // slot row of the warp's first row
-          const bool lane_on = 4 * lane < D;
-#pragma unroll 1
-          for (int i0 = 0; i0 < 32; i0 += 16) {
-            float4 cv[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const bool on = lane_on && ((live >> (i0 + k)) & 1u);
-              if (CBF) {
-                const uint2 hv = on ? __ldcs(reinterpret_cast<const uint2*>(
-                                          reinterpret_cast<const __nv_bfloat16*>(p.cache_O) + (row0 + i0 + k) * D) + lane)
-                                    : make_uint2(0, 0);
-                cv[k] = make_float4(bf16lo(hv.x), bf16hi(hv.x), bf16lo(hv.y), bf16hi(hv.y));
-              } else {
-                cv[k] = on ? __ldcs(reinterpret_cast<const float4*>(p.cache_O + (row0 + i0 + k) * D) + lane)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const int row = 32 * q4 + i0 + k;
-              const float ak = __shfl_sync(0xffffffffu, a, i0 + k), bk = __shfl_sync(0xffffffffu, b, i0 + k);
-              if (lane_on) {
-                float4* o = ot_chunk<DP>(sO, row, lane);
-                float4 ov = *o;
-                ov.x = fmaf(ak, ov.x, bk * cv[k].x);
-                ov.y = fmaf(ak, ov.y, bk * cv[k].y);
-                ov.z = fmaf(ak, ov.z, bk * cv[k].z);
-                ov.w = fmaf(ak, ov.w, bk * cv[k].w);
-                *o = ov;
-              }
+          for (int k = 0; k < 32; ++k) {
+            const int row = 32 * q4 + k;
+            const float ak = __shfl_sync(0xffffffffu, a, k), bk = __shfl_sync(0xffffffffu, b, k);
+            if (lane_on) {
+              const float4 c = ((live >> k) & 1u) ? cv[k] : make_float4(0.f, 0.f, 0.f, 0.f);
+              float4* o = ot_chunk<DP>(sO, row, lane);
+              float4 ov = *o;
+              ov.x = fmaf(ak, ov.x, bk * c.x);
+              ov.y = fmaf(ak, ov.y, bk * c.y);
+              ov.z = fmaf(ak, ov.z, bk * c.z);
+              ov.w = fmaf(ak, ov.w, bk * c.w);
+              *o = ov;
             }
           }
           __syncwarp();
@@ -803,6 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const float m_s = stat_m[st * 128 + r], l_s = stat_l[st * 128 + r];
         mbar_arrive(&bars[C::bStFree + st]);
         if (!warp_wait(&bars[C::bODSeg], cseg & 1, abort_flag, p.status, lim)) goto ep_done;
+        if (warp == kWarpEpi) DT_TR(21, cseg);
         tc_fence_after();
         // O_part -> registers, then hand O_part straight back to the MMA warps
         uint32_t op[DP];
@@ -830,29 +831,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
         const bool track = !WIN && p.err != nullptr &&
                            (p.err_all || seg == (KM == kModeGrouped ? 0 : query_tile<KM>(G, qt).part));
         float e_diff = 0.f, e_norm = 0.f;
+        // 8 columns per step (D = 64, 72, 128 are multiples of 8): two O_tot
+        // chunks, one 32-byte store of the fresh fp32 state when the cache is
+        // 32-byte aligned (rows are D * 4 bytes, a multiple of 32), one 16-byte
+        // store of a bf16 state
 #pragma unroll
-        for (int c = 0; c < D; c += 4) {
-          float old[4], nw[4], x[4];
-          float4* oc = ot_chunk<DP>(sO, r, c / 4);
-          const float4 ov = *oc;
-          old[0] = ov.x; old[1] = ov.y; old[2] = ov.z; old[3] = ov.w;
+        for (int c = 0; c < D; c += 8) {
+          float old[8], nw[8], x[8];
+          float4* oc0 = ot_chunk<DP>(sO, r, c / 4);
+          float4* oc1 = ot_chunk<DP>(sO, r, c / 4 + 1);
+          const float4 o0 = *oc0, o1 = *oc1;
+          old[0] = o0.x; old[1] = o0.y; old[2] = o0.z; old[3] = o0.w;
+          old[4] = o1.x; old[5] = o1.y; old[6] = o1.z; old[7] = o1.w;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 8; ++k) {
             x[k] = u2f(op[c + k]);
             nw[k] = fmaf(a, old[k], b * x[k]);
           }
-          *oc = make_float4(nw[0], nw[1], nw[2], nw[3]);
+          *oc0 = make_float4(nw[0], nw[1], nw[2], nw[3]);
+          *oc1 = make_float4(nw[4], nw[5], nw[6], nw[7]);
           if (valid && track) {
-            float ov[4];
+            float ov[8];
             if (CBF) {
-              const uint2 hv = __ldcs(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.cache_O) + slot * D + c));
+              const uint4 hv = __ldcs(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.cache_O) + slot * D + c));
               ov[0] = bf16lo(hv.x); ov[1] = bf16hi(hv.x); ov[2] = bf16lo(hv.y); ov[3] = bf16hi(hv.y);
+              ov[4] = bf16lo(hv.z); ov[5] = bf16hi(hv.z); ov[6] = bf16lo(hv.w); ov[7] = bf16hi(hv.w);
             } else {
-              const float4 v4 = __ldcs(reinterpret_cast<const float4*>(p.cache_O + slot * D + c));
-              ov[0] = v4.x; ov[1] = v4.y; ov[2] = v4.z; ov[3] = v4.w;
+              const float4 v0 = __ldcs(reinterpret_cast<const float4*>(p.cache_O + slot * D + c));
+              const float4 v1 = __ldcs(reinterpret_cast<const float4*>(p.cache_O + slot * D + c + 4));
+              ov[0] = v0.x; ov[1] = v0.y; ov[2] = v0.z; ov[3] = v0.w;
+              ov[4] = v1.x; ov[5] = v1.y; ov[6] = v1.z; ov[7] = v1.w;
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < 8; ++k) {
               const float nv = x[k] * inv_l;
               e_diff = fmaf(nv - ov[k], nv - ov[k], e_diff);
               e_norm = fmaf(nv, nv, e_norm);
@@ -860,20 +871,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           }
           if (valid) {
             if (!WIN && CBF) {
-              uint2 pk;
+              uint4 pk;
               pk.x = pack_bf16x2(x[0] * inv_l, x[1] * inv_l);
               pk.y = pack_bf16x2(x[2] * inv_l, x[3] * inv_l);
-              __stcs(reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.cache_O) + slot * D + c), pk);
+              pk.z = pack_bf16x2(x[4] * inv_l, x[5] * inv_l);
+              pk.w = pack_bf16x2(x[6] * inv_l, x[7] * inv_l);
+              __stcs(reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.cache_O) + slot * D + c), pk);
             } else if (!WIN) {
-              __stcs(reinterpret_cast<float4*>(p.cache_O + slot * D + c),
-                     make_float4(x[0] * inv_l, x[1] * inv_l, x[2] * inv_l, x[3] * inv_l));
+              const float4 f0 = make_float4(x[0] * inv_l, x[1] * inv_l, x[2] * inv_l, x[3] * inv_l);
+              const float4 f1 = make_float4(x[4] * inv_l, x[5] * inv_l, x[6] * inv_l, x[7] * inv_l);
+              float* dst = p.cache_O + slot * D + c;
+              if (p.cache_v8) {
+                st_cs_v8(dst, f0, f1);
+              } else {
+                __stcs(reinterpret_cast<float4*>(dst), f0);
+                __stcs(reinterpret_cast<float4*>(dst + 4), f1);
+              }
             } else if (make_r) {
-              float4 v;
-              v.x = nw[0] * inv_new - old[0] * inv_tot;
-              v.y = nw[1] * inv_new - old[1] * inv_tot;
-              v.z = nw[2] * inv_new - old[2] * inv_tot;
-              v.w = nw[3] * inv_new - old[3] * inv_tot;
-              __stcs(reinterpret_cast<float4*>(p.R + ((size_t)h * G.S + qrow) * D + c), v);
+              float* dst = p.R + ((size_t)h * G.S + qrow) * D + c;
+              __stcs(reinterpret_cast<float4*>(dst), make_float4(nw[0] * inv_new - old[0] * inv_tot,
+                                                                nw[1] * inv_new - old[1] * inv_tot,
+                                                                nw[2] * inv_new - old[2] * inv_tot,
+                                                                nw[3] * inv_new - old[3] * inv_tot));
+              __stcs(reinterpret_cast<float4*>(dst + 4), make_float4(nw[4] * inv_new - old[4] * inv_tot,
+                                                                    nw[5] * inv_new - old[5] * inv_tot,
+                                                                    nw[6] * inv_new - old[6] * inv_tot,
+                                                                    nw[7] * inv_new - old[7] * inv_tot));
             }
           }
         }
@@ -891,6 +914,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
           }
         }
         if (!WIN && valid) __stcs(p.cache_L + slot, nonempty ? (m_s + lg2(l_s)) * kLn2 : kNegInf);
+        if (warp == kWarpEpi) DT_TR(22, cseg);
         if (have || nonempty) { m_tot = m_new; l_tot = l_new; }
         have = have || nonempty;
         ++cseg;

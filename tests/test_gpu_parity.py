@@ -224,6 +224,32 @@ def test_output_guard_bands_untouched():
     assert torch.isfinite(sess.O.float()).all()
 
 
+@pytest.mark.parametrize("D", [72, 128])
+def test_cache_alignment_16_matches_32(D):
+    """A state cache that starts on a 16-byte (not 32-byte) boundary takes
+    the 16-byte store path for fresh states; outputs, LSEs and every cache
+    byte equal those of a 32-byte-aligned cache."""
+    H, S, P = 2, 1100, 4
+    q, k, v = wl.InputStream(H, S, D, 0.05, seed=21).next_step()
+    q2, k2, v2 = wl.InputStream(H, S, D, 0.05, seed=22).next_step()
+    runs = []
+    for offset in (0, 4):                          # floats: 0 or 16 bytes past a 256-byte boundary
+        sess = Session(H, S, D, P, mode=dt.DT_MODE_PROXIMITY, reuse_per_row=2)
+        n = sess.cache_O.numel()
+        big = torch.zeros(n + 8, dtype=torch.float32, device="cuda")
+        sess.cache_O = big[offset:offset + n].view(sess.cache_O.shape)
+        assert (sess.cache_O.data_ptr() % 32 == 0) == (offset == 0)
+        sess.set_inputs(q, k, v)
+        sess.step(1)
+        sess.set_inputs(q2, k2, v2)
+        sess.step(2)
+        sess.check()
+        runs.append((sess.O.clone(), sess.L.clone(), sess.cache_O.clone(), sess.cache_L.clone()))
+    for a, b in zip(*runs):
+        assert torch.equal(a.view(torch.int32) if a.dtype == torch.float32 else a.view(torch.int16),
+                           b.view(torch.int32) if b.dtype == torch.float32 else b.view(torch.int16))
+
+
 # ------------------------------------------------------------------ window mode
 
 def run_window_schedule(H, S, D, W, steps, inputs, heads=None, rows=None):
