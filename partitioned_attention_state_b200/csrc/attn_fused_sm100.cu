@@ -927,19 +927,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
       if (valid) {
         const float inv = (have && l_tot > 0.f) ? 1.f / l_tot : 0.f;
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.O) + ((size_t)h * G.S + qrow) * D;
-        const float* rr = p.R + ((size_t)h * G.S + qrow) * D;
-#pragma unroll 2
-        for (int c = 0; c < D; c += 4) {
-          const float4 ov = *ot_chunk<DP>(sO, r, c / 4);
-          float v0 = ov.x * inv, v1 = ov.y * inv, v2 = ov.z * inv, v3 = ov.w * inv;
-          if (use_r) {
-            const float4 rv = __ldcs(reinterpret_cast<const float4*>(rr + c));
-            v0 += rv.x; v1 += rv.y; v2 += rv.z; v3 += rv.w;
+        if (WIN && use_r) {
+          // the residual row is read whole before any output store (one
+          // memory round trip); 8 output columns (16 bytes of bf16) per store
+          const float4* rr = reinterpret_cast<const float4*>(p.R + ((size_t)h * G.S + qrow) * D);
+          float4 rv[D / 4];
+#pragma unroll
+          for (int c = 0; c < D / 4; ++c) rv[c] = __ldcs(rr + c);
+#pragma unroll
+          for (int c = 0; c < D; c += 8) {
+            const float4 o0 = *ot_chunk<DP>(sO, r, c / 4), o1 = *ot_chunk<DP>(sO, r, c / 4 + 1);
+            const float4 r0 = rv[c / 4], r1 = rv[c / 4 + 1];
+            uint4 pk;
+            pk.x = pack_bf16x2(fmaf(o0.x, inv, r0.x), fmaf(o0.y, inv, r0.y));
+            pk.y = pack_bf16x2(fmaf(o0.z, inv, r0.z), fmaf(o0.w, inv, r0.w));
+            pk.z = pack_bf16x2(fmaf(o1.x, inv, r1.x), fmaf(o1.y, inv, r1.y));
+            pk.w = pack_bf16x2(fmaf(o1.z, inv, r1.z), fmaf(o1.w, inv, r1.w));
+            __stcs(reinterpret_cast<uint4*>(dst + c), pk);
           }
-          uint2 pk;
-          pk.x = pack_bf16x2(v0, v1);
-          pk.y = pack_bf16x2(v2, v3);
-          __stcs(reinterpret_cast<uint2*>(dst + c), pk);
+        } else {
+#pragma unroll 2
+          for (int c = 0; c < D; c += 4) {
+            const float4 ov = *ot_chunk<DP>(sO, r, c / 4);
+            uint2 pk;
+            pk.x = pack_bf16x2(ov.x * inv, ov.y * inv);
+            pk.y = pack_bf16x2(ov.z * inv, ov.w * inv);
+            __stcs(reinterpret_cast<uint2*>(dst + c), pk);
+          }
         }
         __stcs(p.L + (size_t)h * G.S + qrow, (have && l_tot > 0.f) ? (m_tot + lg2(l_tot)) * kLn2 : kNegInf);
       }
