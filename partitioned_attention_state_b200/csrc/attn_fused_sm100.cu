@@ -945,14 +945,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_partial_fused_kernel(const _
             pk.w = pack_bf16x2(fmaf(o1.z, inv, r1.z), fmaf(o1.w, inv, r1.w));
             __stcs(reinterpret_cast<uint4*>(dst + c), pk);
           }
-        } else {
+        } else {   // 8 output columns (16 bytes of bf16) per store
 #pragma unroll 2
-          for (int c = 0; c < D; c += 4) {
-            const float4 ov = *ot_chunk<DP>(sO, r, c / 4);
-            uint2 pk;
-            pk.x = pack_bf16x2(ov.x * inv, ov.y * inv);
-            pk.y = pack_bf16x2(ov.z * inv, ov.w * inv);
-            __stcs(reinterpret_cast<uint2*>(dst + c), pk);
+          for (int c = 0; c < D; c += 8) {
+            const float4 o0 = *ot_chunk<DP>(sO, r, c / 4), o1 = *ot_chunk<DP>(sO, r, c / 4 + 1);
+            uint4 pk;
+            pk.x = pack_bf16x2(o0.x * inv, o0.y * inv);
+            pk.y = pack_bf16x2(o0.z * inv, o0.w * inv);
+            pk.z = pack_bf16x2(o1.x * inv, o1.y * inv);
+            pk.w = pack_bf16x2(o1.z * inv, o1.w * inv);
+            __stcs(reinterpret_cast<uint4*>(dst + c), pk);
           }
         }
         __stcs(p.L + (size_t)h * G.S + qrow, (have && l_tot > 0.f) ? (m_tot + lg2(l_tot)) * kLn2 : kNegInf);
