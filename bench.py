@@ -669,7 +669,12 @@ def main():
                          "peak": peak_tf, "peak_kind": f"{pk_kind} bf16 dense (burst)", "unit": "TFLOP/s",
                          "frac": achieved / peak_tf, "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
                          "nominal_peak": NOMINAL_BF16_TFLOPS, "traffic": traffic, "kernel_ms": kern_ms,
-                         "flops_per_launch": flops},
+                         "flops_per_launch": flops,
+                         # the step runs back to back under the power cap: the measured
+                         # seconds-long GEMM figure, when present, as a second denominator
+                         "sustained_peak": pk.get("bf16_tflops_sustained"),
+                         "frac_of_sustained": (achieved / float(pk["bf16_tflops_sustained"])
+                                               if pk.get("bf16_tflops_sustained") else None)},
             "gpu_launches": args.steps,
             "clocks": clocks,
             "e2e": e2e,
