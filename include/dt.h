@@ -248,7 +248,9 @@ DT_API int dt_anchor_update(const dt_plan_params* p, dt_anchor_state* a, const i
  *   d_status    int32 device status word (see conventions)
  * The host validates shapes and alignment before any launch.  One launch.
  * Partition mode supports at most 64 key sets (DT_ERR_UNSUPPORTED above);
- * d_plan must be 16-byte aligned like every other pointer. */
+ * d_plan must be 16-byte aligned like every other pointer.  A cache_O that
+ * starts on a 32-byte boundary lets the kernel store fresh fp32 states 32
+ * bytes per instruction (results are identical either way). */
 DT_API int dt_attn_partial_fused(const dt_plan_params* p, const uint8_t* d_plan,
                           const void* Q, const void* K, const void* V,
                           float* cache_O, float* cache_L, float* R,
