@@ -513,3 +513,43 @@ def test_anchor_calls_validated():
     pw = dt.params(1, 1024, 64, 1, dt.DT_MODE_WINDOW, 0, 64, 1)
     assert lib.dt_attn_partial_fused_tracked(ctypes.byref(pw), *([None] * 11), 0, None) == dt.DT_ERR_INVALID
     assert lib.dt_plan_build(ctypes.byref(p), None, ctypes.byref(plan)) == dt.DT_ERR_INVALID      # needs its state
+
+
+def test_plan_matches_oracle_on_random_geometry():
+    """Seeded random geometries (ragged sequences, partition counts up to 24,
+    groups of 1 to 5, every head dim), each through an anchor, two reuse steps
+    with different r, an all-reuse step and an explicit plan: plans, counts
+    and stamps bit-exact with the oracle's planner."""
+    rng = np.random.Generator(np.random.PCG64(2024))
+    for _ in range(40):
+        S = int(rng.integers(1, 6000))
+        P = int(rng.integers(1, 25))
+        D = int(rng.choice([64, 72, 128]))
+        H = int(rng.integers(1, 4))
+        g = int(rng.choice([0, 0, 1, 2, 3, 5]))
+        n_sets = P if g == 0 else -(-P // g)
+        if n_sets + (1 if g else 0) > 64:
+            continue
+        p = dt.params(H, S, D, P, dt.DT_MODE_PROXIMITY, 0, 0, 1, g)
+        nqt, nseg = dt.dt_plan_geometry(p)
+        st = np.full((nqt, nseg), -1, np.int32)
+        r1, r2 = (int(rng.integers(0, max(1, n_sets))) for _ in range(2))
+        _, _, st = run_both(orc.MODE_PROXIMITY, H, S, D, P, 1, r=r1, stamps=st, group=g)
+        _, _, st = run_both(orc.MODE_PROXIMITY, H, S, D, P, 2, r=r1, stamps=st, group=g)
+        _, _, st = run_both(orc.MODE_PROXIMITY, H, S, D, P, 3, r=r2, stamps=st, group=g)
+        _, _, st = run_both(orc.MODE_ALL_REUSE, H, S, D, P, 4, stamps=st, group=g)
+        ex = (rng.random((nqt, nseg)) < 0.5).astype(np.uint8)
+        run_both(orc.MODE_EXPLICIT, H, S, D, P, 5, stamps=st, explicit=ex, group=g)
+
+
+def test_window_plan_matches_oracle_on_random_geometry():
+    rng = np.random.Generator(np.random.PCG64(2025))
+    for _ in range(30):
+        S = int(rng.integers(1, 9000))
+        W = int(rng.integers(1, 2 * S + 2))
+        H, D = int(rng.integers(1, 4)), int(rng.choice([64, 72, 128]))
+        p = dt.params(H, S, D, 1, dt.DT_MODE_WINDOW, 0, W, 1)
+        nqt, nseg = dt.dt_plan_geometry(p)
+        st = np.full((nqt, nseg), -1, np.int32)
+        for step in (1, 2, 3):
+            _, _, st = run_both(orc.MODE_WINDOW, H, S, D, 1, step, window=W, stamps=st)
