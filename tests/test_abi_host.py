@@ -453,7 +453,8 @@ def _sum_errors(err, plan, stamps_before):
     return diff, norm
 
 
-@pytest.mark.parametrize("S,P,g,rho", [(4096, 16, 0, 0.5), (4096, 16, 4, 0.4), (1800, 12, 0, 0.3), (2600, 7, 2, 0.75)])
+@pytest.mark.parametrize("S,P,g,rho", [(4096, 16, 0, 0.5), (4096, 16, 4, 0.4), (1800, 12, 0, 0.3), (2600, 7, 2, 0.75),
+                                        (777, 1, 0, 0.5), (3001, 5, 0, 1.0), (5000, 24, 5, 0.0), (650, 20, 3, 0.6)])
 def test_anchor_planner_matches_oracle(S, P, g, rho):
     """dt_plan_build_anchor / dt_anchor_update against the oracle's
     anchor_plan / anchor_update on random measurements over 10 steps,
