@@ -554,3 +554,51 @@ def test_window_plan_matches_oracle_on_random_geometry():
         st = np.full((nqt, nseg), -1, np.int32)
         for step in (1, 2, 3):
             _, _, st = run_both(orc.MODE_WINDOW, H, S, D, 1, step, window=W, stamps=st)
+
+
+def test_plan_parameters_fuzzed():
+    """Seeded random parameter sets, valid and invalid (negative, zero, huge
+    or inconsistent fields, every mode): the host planner either rejects them
+    with a status code or builds a plan whose counts add up, and never
+    crashes; accepted all-compute plans match the oracle's."""
+    import ctypes
+    lib = dt.load()
+    rng = np.random.Generator(np.random.PCG64(77))
+    pick = lambda *vals: int(rng.choice(vals))
+    accepted = 0
+    for _ in range(400):
+        H = pick(-1, 0, 1, 2, 3, 1 << 20)
+        S = pick(-5, 0, 1, 127, 128, 129, 1000, 4097, 1 << 30)
+        D = pick(0, 8, 64, 72, 100, 128, 256)
+        P = pick(-1, 0, 1, 3, 16, 64, 65, 200)
+        mode = pick(-1, 0, 1, 2, 3, 4, 5, 6, 7, 99)
+        r = pick(-2, 0, 1, 7, 15, 64)
+        window = pick(-1, 0, 1, 64, 1000, 1 << 30)
+        step = pick(-1, 0, 1, 2, 5)
+        group = pick(-1, 0, 1, 3, 8, 100)
+        p = dt.params(H, S, D, P, mode, r, window, step, group)
+        nqt, nseg = ctypes.c_int32(), ctypes.c_int32()
+        rc = lib.dt_plan_geometry(ctypes.byref(p), ctypes.byref(nqt), ctypes.byref(nseg))
+        if rc != dt.DT_OK:
+            assert rc in (dt.DT_ERR_INVALID, dt.DT_ERR_UNSUPPORTED), rc
+            continue
+        if nqt.value * nseg.value > 1 << 22:                 # huge but valid: skip the build
+            continue
+        plan = np.zeros((max(nqt.value, 1), max(nseg.value, 1)), np.uint8)
+        st = np.full(plan.shape, 1, np.int32)                # every slot cached at step 1
+        out = dt.Plan()
+        out.plan = plan.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+        out.stamps = st.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        ex = np.zeros(plan.shape, np.uint8)
+        rc = lib.dt_plan_build(ctypes.byref(p), ex.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), ctypes.byref(out))
+        if rc != dt.DT_OK:
+            assert rc in (dt.DT_ERR_INVALID, dt.DT_ERR_UNSUPPORTED, dt.DT_ERR_CACHE_EMPTY), rc
+            continue
+        accepted += 1
+        assert out.computed_blocks >= 0 and out.skipped_blocks >= 0
+        assert set(np.unique(plan[: nqt.value, : nseg.value])) <= {0, 1}
+        if mode == dt.DT_MODE_ALL_COMPUTE and group == 0 and H * S < 1 << 16:
+            want, counts, _ = orc.build_plan(orc.MODE_ALL_COMPUTE, H, S, D, P, step)
+            np.testing.assert_array_equal(plan[: nqt.value, : nseg.value], want)
+            assert out.computed_blocks == counts["computed_blocks"]
+    assert accepted > 20
